@@ -1,0 +1,201 @@
+/*
+ * pa.h: C ABI of libpa.so, paged-KV attention on NVIDIA B200 (sm_100a).
+ *
+ * The method. The KV cache is split into fixed-size blocks of 16 tokens that
+ * live anywhere in one physical pool. Each sequence keeps a table that maps
+ * its logical blocks to physical ones. Attention reads K/V block by block
+ * through that table ("vLLM and PagedAttention", ai.zenoagi.com, §2 "The
+ * PagedAttention Solution" and "Reworking the Attention Computation";
+ * "vLLM — PagedAttention and Continuous Batching", s-samarth.github.io, §2.2
+ * and §2.4). A sequence takes a new block only when its last one is full, so
+ * only the last block can be partly filled ("How vLLM Works?",
+ * peterindia.net, §03).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are caller-owned DEVICE memory on the current CUDA
+ *    device. They are row-major and contiguous, and 16-byte aligned. The
+ *    library allocates nothing and keeps no state except a cached SM count
+ *    per device and one device status word (pa_get_status).
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream. Calls only enqueue work, never synchronize (except
+ *    pa_get_status) and never allocate, so they can be captured in CUDA graphs.
+ *  - Element type of q, k, v, the caches and out is shape->dtype. The
+ *    tables, lengths and slot mapping are int32/int64 as declared.
+ *  - Return value: PA_OK, or a negative pa_error. On an argument error
+ *    nothing is launched. PA_ERR_CUDA means a launch failed; the CUDA error
+ *    stays readable with cudaGetLastError().
+ *  - Bad data inside device buffers cannot be checked on the host without a
+ *    sync: a table entry outside the pool, a slot outside the pool, a
+ *    context length over the table's capacity. The kernels check these as
+ *    they read them. A bad item is skipped (never dereferenced) and a flag is
+ *    set in the device status word (PA_STATUS_*). Outputs that depended on
+ *    it are then unspecified. Read the word with pa_get_status().
+ *
+ * Layouts (B = sequences, H = query heads, Hk = KV heads, D = head_dim,
+ * NB = pool blocks, S = block size = 16, MB = table width):
+ *   k_cache, v_cache : [NB][S][Hk][D]   (the kernel sketch's
+ *                      [num_blocks, block_size, num_heads, d_head] comment
+ *                      in "vLLM and PagedAttention" §2, with KV heads)
+ *   block_tables     : int32 [B][MB], physical block of logical block i
+ *   context_lens     : int32 [B], tokens in the sequence INCLUDING this
+ *                      step's new ones (the cache write comes first)
+ *   q, out           : [tokens][H][D]. The sketch's output comment
+ *                      "[seq_len, d_model]" is read as this.
+ *   k, v (new tokens): [T][Hk][D]
+ * Query head h uses KV head h / (H / Hk) (contiguous groups).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+#define PA_BLOCK_SIZE 16
+
+typedef enum {
+    PA_DTYPE_F32 = 0,  /* IEEE fp32 */
+    PA_DTYPE_BF16 = 1, /* bfloat16 */
+} pa_dtype;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARGUMENT = -1, /* null pointer, negative size, inconsistent sizes */
+    PA_ERR_UNSUPPORTED = -2,      /* shape/dtype combination not compiled in */
+    PA_ERR_ALIGNMENT = -3,        /* a pointer is not 16-byte aligned */
+    PA_ERR_WORKSPACE = -4,        /* workspace missing or smaller than pa_decode_workspace_bytes */
+    PA_ERR_CUDA = -5,             /* a CUDA runtime call or launch failed */
+    PA_ERR_DEVICE = -6,           /* no usable device, or not an sm_100 device */
+} pa_error;
+
+/* Flags of the device status word (OR-ed together). */
+#define PA_STATUS_BAD_BLOCK_ID 0x1u   /* table entry outside [0, NB) */
+#define PA_STATUS_BAD_SLOT 0x2u       /* slot_mapping entry >= NB * 16 */
+#define PA_STATUS_BAD_CONTEXT 0x4u    /* context length < 0, > MB * 16, or > max_context_len */
+#define PA_STATUS_WAIT_TIMEOUT 0x8u   /* a bounded wait on an async copy gave up */
+#define PA_STATUS_BAD_QUERY 0x10u     /* prefill: q_len > context_len or cu_q_lens not increasing */
+
+typedef struct {
+    int32_t num_heads;    /* H, query heads */
+    int32_t num_kv_heads; /* Hk, KV heads; H % Hk == 0 and H / Hk in {1, 2, 4, 8} */
+    int32_t head_dim;     /* D: 64 or 128 */
+    int32_t block_size;   /* tokens per block: must be 16 */
+    int64_t num_blocks;   /* NB, blocks in the pool */
+    int32_t dtype;        /* pa_dtype */
+} pa_shape;
+
+/*
+ * pa_reshape_and_cache: append this step's new tokens to the cache.
+ *
+ * For every t in [0, num_tokens) with slot_mapping[t] >= 0, copy the [Hk][D]
+ * row k[t] to k_cache viewed as [NB*16][Hk][D] at row slot_mapping[t], and
+ * the same for v. A slot is physical_block * 16 + row. A negative slot means
+ * padding and that token is skipped. Every other byte of the caches is left
+ * alone and the copy is bit-exact. This is the on-demand slot fill of
+ * "vLLM and PagedAttention" §2 "The PagedAttention Solution" ("the 7th block
+ * is only requested when the 100th token is generated") and of
+ * "How vLLM Works?" §03.
+ *
+ *   k, v         : [num_tokens][Hk][D] device
+ *   k_cache,
+ *   v_cache      : [NB][16][Hk][D] device, updated in place
+ *   slot_mapping : int64 [num_tokens] device
+ * Duplicate non-negative slots in one call: which token lands is unspecified.
+ * A slot >= NB*16 is skipped and sets PA_STATUS_BAD_SLOT.
+ * num_tokens == 0 is a no-op.
+ */
+int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int64_t num_tokens, const pa_shape *shape,
+                         void *stream);
+
+/*
+ * pa_decode_workspace_bytes: scratch size pa_decode needs for these sizes
+ * and this partition_tokens (0 = automatic), on the current device. It is 0
+ * when the single-pass kernel covers every sequence. Negative on bad
+ * arguments.
+ */
+int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int32_t partition_tokens,
+                                  const pa_shape *shape);
+
+/*
+ * pa_decode: one query token per sequence attends over its whole paged
+ * context (decode-time PagedAttention; "vLLM and PagedAttention" §2
+ * "Reworking the Attention Computation": K/V are loaded block by block and
+ * each block's share is folded into the result).
+ *
+ *   out[b][h][:] = sum_p softmax_p(scale * q[b][h] . K_b[p]) V_b[p],
+ *   p over 0 .. context_lens[b]-1, K_b[p] = k_cache[block_tables[b][p/16]][p%16][h/(H/Hk)]
+ *
+ *   out          : [B][H][D] device
+ *   q            : [B][H][D] device
+ *   block_tables : int32 [B][max_blocks_per_seq] device; entries past
+ *                  ceil(context_lens[b]/16) are never read
+ *   context_lens : int32 [B] device; 0 gives an all-zero output row
+ *   max_context_len : host-side upper bound of context_lens (no device read);
+ *                  it sizes the grid and the workspace. A device length above
+ *                  it is clamped and sets PA_STATUS_BAD_CONTEXT.
+ *   scale        : softmax scale (the sketch has none; typically 1/sqrt(D))
+ *   partition_tokens : 0 = automatic. Otherwise tokens per split-context
+ *                  partition, a multiple of 64 and >= 64. A context longer
+ *                  than one partition is split. Each partition writes
+ *                  (max, sum, unnormalised O) to the workspace and a second
+ *                  kernel merges them.
+ *   workspace    : device scratch of >= pa_decode_workspace_bytes(...) bytes,
+ *                  16-byte aligned. It may be NULL when that size is 0. Its
+ *                  contents need no initialisation, and calls that overlap on
+ *                  the GPU must not share one.
+ * Accumulation is fp32 whatever the dtype. bf16 output is rounded once, to
+ * nearest even.
+ */
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+              float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
+              const pa_shape *shape, void *stream);
+
+/*
+ * pa_prefill_chunk: causal attention for chunks of query tokens placed at a
+ * context offset (chunked prefill: "vLLM — PagedAttention and Continuous
+ * Batching" §5; "How vLLM Works?" §04). The chunk's K/V must already be in
+ * the cache (pa_reshape_and_cache first).
+ *
+ * Sequence b owns query rows cu_q_lens[b] .. cu_q_lens[b+1]-1. Its chunk
+ * length is q_len = cu_q_lens[b+1] - cu_q_lens[b] and its offset is
+ * o = context_lens[b] - q_len. Row j of the chunk sits at absolute position
+ * o + j and attends to keys 0 .. o + j (inclusive) of the paged context.
+ *
+ *   out, q       : [num_q_tokens][H][D] device, num_q_tokens = cu_q_lens[B]
+ *   cu_q_lens    : int32 [B + 1] device, non-decreasing, cu_q_lens[0] = 0
+ *   context_lens : int32 [B] device, >= q_len
+ *   max_q_len    : host-side upper bound of every q_len (sizes the grid)
+ * bf16 only, D = 128 only. Runs on the tcgen05 tensor cores with fp32
+ * accumulation in tensor memory. Returns PA_ERR_UNSUPPORTED otherwise.
+ */
+int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *cu_q_lens,
+                     const int32_t *context_lens, int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens,
+                     float scale, const pa_shape *shape, void *stream);
+
+/*
+ * pa_get_status: synchronize `stream`, copy the device status word of the
+ * current device to *status (PA_STATUS_* flags, 0 = clean), then clear it.
+ */
+int pa_get_status(uint32_t *status, void *stream);
+
+/* Static text for a pa_error code. */
+const char *pa_strerror(int code);
+
+/* cudaError_t code of the last PA_ERR_CUDA returned on this host thread (0 if none). */
+int pa_last_cuda_error(void);
+
+/* PA_ABI_VERSION of the loaded library. */
+int pa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

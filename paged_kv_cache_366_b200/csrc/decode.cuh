@@ -1,0 +1,404 @@
+// Decode-time paged attention (one query token per sequence), sm_100a.
+//
+// What it computes ("vLLM and PagedAttention", ai.zenoagi.com, §2 "Reworking
+// the Attention Computation"): for each sequence b and query head h,
+//   out[b][h] = softmax(scale * q[b][h] . K_b^T) V_b
+// where row p of K_b/V_b sits in physical block block_tables[b][p / 16] at row
+// p % 16. Blocks are loaded one by one and each block's share is folded into
+// a running result. That is online softmax: a running max m, a running sum l
+// and an accumulator O rescaled by exp(m_old - m_new) whenever m grows.
+//
+// How it runs on B200:
+//  * Grid (partition, KV head, sequence). A CTA owns one KV head of one
+//    sequence over one partition of the context (split-context pass).
+//    Sequences longer than a partition also write (m, l, O) partials, and
+//    decode_reduce_kernel merges them.
+//  * Every query head of the KV head's group (G = H / Hk of them) reads each
+//    loaded block from shared memory, so K/V cross HBM once per KV head.
+//  * The 4 warps of a CTA take the partition's blocks round-robin. Each warp
+//    streams its own blocks through an NSTAGE-deep shared-memory ring. A
+//    block's 16 K rows and 16 V rows are fetched by 32 TMA bulk copies (one
+//    per lane, a 256-byte row each at D=128 bf16) into a ring slot, and an
+//    mbarrier counts the bytes. Fetches run NSTAGE blocks ahead, so the
+//    table entry, the HBM fetch and the math of different blocks overlap.
+//  * Lanes own column slices of a row made of CH 16-byte chunks (CH = 2, or 1
+//    for groups of 8 heads to bound registers), interleaved so shared-memory
+//    reads are conflict free. L = row_bytes / (16 * CH) lanes cover a row and RS = 32 / L rows are processed per step. q.k
+//    partial sums are folded across the L lanes with a transpose-reduce
+//    (each shuffle step halves the values per lane). Softmax runs in fp32
+//    (exp2 with scale * log2(e) folded into q). P.V uses packed two-wide
+//    fp32 FMAs.
+//  * Each warp keeps its own (m, l, O). At the end the warps merge through
+//    shared memory (reusing the ring).
+#pragma once
+
+#include <math_constants.h>
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeThreads = 32 * kDecodeWarps;
+
+template <typename T, int D, int G>
+struct DecodeCfg {
+    static constexpr int E = sizeof(T);
+    static constexpr int R = D * E;                        // bytes of one token row of one KV head
+    static constexpr int CH = G >= 8 ? 1 : 2;              // 16-byte chunks a lane owns per row
+    static constexpr int L = R / (16 * CH);                // lanes covering one row
+    static constexpr int RS = 32 / L;                      // rows per warp step
+    static constexpr int STEPS = kBlockSize / RS;          // steps per block
+    static constexpr int VE = 16 / E;                      // elements per 16-byte chunk
+    static constexpr int EPL = CH * VE;                    // elements per lane per row
+    static constexpr int STAGE_BYTES = 2 * kBlockSize * R; // K and V of one block
+    static constexpr int NSTAGE = STAGE_BYTES <= 8192 ? 3 : 2;
+    static constexpr int WARP_RING = NSTAGE * STAGE_BYTES;
+    static constexpr int RING_BYTES = kDecodeWarps * WARP_RING;
+    static constexpr int NPART = STEPS * G;                // q.k partials per lane per block
+    static constexpr int NFIN = NPART >= L ? NPART / L : 1; // fully reduced scores per lane
+    static constexpr int ENT = (kBlockSize * G) / 32 > 0 ? (kBlockSize * G) / 32 : 1;
+    static constexpr int RED_BYTES = kDecodeWarps * RS * G * D * 4;
+    static constexpr int BIG = RING_BYTES > RED_BYTES ? RING_BYTES : RED_BYTES;
+    static constexpr int OFF_BAR = BIG;
+    static constexpr int OFF_S = OFF_BAR + kDecodeWarps * NSTAGE * 8;
+    static constexpr int OFF_ML = OFF_S + kDecodeWarps * kBlockSize * G * 4;
+    static constexpr int SMEM = OFF_ML + 2 * kDecodeWarps * G * 4;
+    static_assert(R % (16 * CH) == 0 && L >= 1 && L <= 32 && 32 % L == 0, "row must split into lane slices");
+    static_assert(kBlockSize % RS == 0, "rows per step must divide the block");
+    static_assert(32 % G == 0 && G <= 8, "group size");
+};
+
+// Sum N values per lane across groups of lanes that differ in the bits of
+// OFF, OFF/2, ..., 1. Every step sends half of the remaining values to the
+// partner lane and keeps the other half, so the lane ends with
+// max(1, N / (2*OFF)) fully summed values. `base` gets the index (into the
+// original N) of the first one.
+template <int N, int OFF>
+struct TransposeReduce {
+    template <int NA>
+    __device__ __forceinline__ static void run(float (&v)[NA], int lane, int &base) {
+        if constexpr (OFF == 0) {
+            return;
+        } else if constexpr (N > 1) {
+            constexpr int H = N / 2;
+            const bool upper = (lane & OFF) != 0;
+#pragma unroll
+            for (int i = 0; i < H; ++i) {
+                const float send = upper ? v[i] : v[i + H];
+                const float keep = upper ? v[i + H] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+            }
+            if (upper) base += H;
+            TransposeReduce<H, OFF / 2>::run(v, lane, base);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            TransposeReduce<1, OFF / 2>::run(v, lane, base);
+        }
+    }
+};
+
+struct DecodeParams {
+    void *out;
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int *block_tables;
+    const int *context_lens;
+    float *ws_o;  // [B][H][max_parts][D]
+    float *ws_m;  // [B][H][max_parts]
+    float *ws_l;  // [B][H][max_parts]
+    long long num_blocks;
+    int max_blocks_per_seq;
+    int num_heads;
+    int num_kv_heads;
+    int max_context_len;
+    int part_tokens;
+    int max_parts;
+    float scale_log2;  // softmax scale * log2(e)
+};
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams prm) {
+    using C = DecodeCfg<T, D, G>;
+    const int p = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
+    const int c = clamp_context(__ldg(prm.context_lens + b), cap, p == 0 && hk == 0 && threadIdx.x == 0);
+    const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
+    if (p >= parts) return;
+
+    const int part_blocks = prm.part_tokens / kBlockSize;
+    const int nblk_seq = (c + kBlockSize - 1) / kBlockSize;
+    const int blk0 = p * part_blocks;
+    const int nb_cta = max(0, min(nblk_seq - blk0, part_blocks));
+    const int last_valid = c - (nblk_seq - 1) * kBlockSize;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int rg = lane / C::L, j = lane % C::L;
+
+    unsigned char *ring = smem + warp * C::WARP_RING;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bars = smem_addr(smem + C::OFF_BAR) + warp * C::NSTAGE * 8;
+    float *s_buf = reinterpret_cast<float *>(smem + C::OFF_S) + warp * kBlockSize * G;
+
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < C::NSTAGE; ++s) mbar_init(bars + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // This warp's blocks: partition block warp + k * kDecodeWarps, k < nb_w.
+    const int nb_w = nb_cta > warp ? (nb_cta - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq + blk0;
+    int tbl = lane < nb_w ? __ldg(trow + warp + lane * kDecodeWarps) : 0;
+    uint32_t bad_mask = 0;
+    const T *kc = static_cast<const T *>(prm.k_cache);
+    const T *vc = static_cast<const T *>(prm.v_cache);
+
+    auto issue = [&](int k) {
+        if (k >= 32 && (k & 31) == 0)
+            tbl = k + lane < nb_w ? __ldg(trow + warp + (k + lane) * kDecodeWarps) : 0;
+        int pb = __shfl_sync(0xffffffffu, tbl, k & 31);
+        const int s = k % C::NSTAGE;
+        if (pb < 0 || pb >= prm.num_blocks) {
+            if (lane == 0) flag_status(PA_STATUS_BAD_BLOCK_ID);
+            pb = 0;
+            bad_mask |= 1u << s;
+        } else {
+            bad_mask &= ~(1u << s);
+        }
+        const uint32_t bar = bars + 8 * s;
+        if (lane == 0) mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+        __syncwarp();
+        const int row = lane & (kBlockSize - 1);
+        const T *src = (lane < kBlockSize ? kc : vc) +
+                       ((static_cast<size_t>(pb) * kBlockSize + row) * prm.num_kv_heads + hk) * D;
+        const uint32_t dst = ring_s + s * C::STAGE_BYTES + (lane < kBlockSize ? 0 : kBlockSize * C::R) + row * C::R;
+        bulk_g2s(dst, src, C::R, bar);
+    };
+
+    // Queries of the group, pre-scaled by scale * log2(e).
+    float qf[G][C::EPL];
+    {
+        const T *qb = static_cast<const T *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int ch = 0; ch < C::CH; ++ch) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + (ch * C::L + j) * C::VE));
+                Widen<T>::apply(raw, &qf[g][ch * C::VE]);
+#pragma unroll
+                for (int e = 0; e < C::VE; ++e) qf[g][ch * C::VE + e] *= prm.scale_log2;
+            }
+    }
+
+    float acc[G][C::EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < C::EPL; ++e) acc[g][e] = 0.f;
+    float m_own = -CUDART_INF_F;  // running max of head lane % G (log2 domain)
+    float l_own = 0.f;            // this lane's share of that head's running sum
+
+    int issued = 0;
+    for (; issued < min(C::NSTAGE, nb_w); ++issued) issue(issued);
+
+    int k = 0;
+    bool failed = false;
+    for (; k < nb_w; ++k) {
+        const int s = k % C::NSTAGE;
+        const bool landed = mbar_wait(bars + 8 * s, (k / C::NSTAGE) & 1);
+        if (!__all_sync(0xffffffffu, landed)) {
+            failed = true;
+            break;
+        }
+        const int lblk = blk0 + warp + k * kDecodeWarps;
+        const int n_valid = ((bad_mask >> s) & 1u) ? 0 : (lblk == nblk_seq - 1 ? last_valid : kBlockSize);
+        const unsigned char *kb = ring + s * C::STAGE_BYTES;
+        const unsigned char *vb = kb + kBlockSize * C::R;
+
+        // ---- scores: q . k for the G heads and this lane's rows
+        float part[C::NPART];
+#pragma unroll
+        for (int st = 0; st < C::STEPS; ++st) {
+            const int row = st * C::RS + rg;
+            float kf[C::EPL];
+#pragma unroll
+            for (int ch = 0; ch < C::CH; ++ch) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(kb + row * C::R + (ch * C::L + j) * 16);
+                Widen<T>::apply(raw, &kf[ch * C::VE]);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int e = 0; e < C::EPL; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1]);
+                part[st * G + g] = a0 + a1;
+            }
+        }
+        int base = 0;
+        TransposeReduce<C::NPART, C::L / 2>::run(part, lane, base);
+#pragma unroll
+        for (int f = 0; f < C::NFIN; ++f) {
+            const int idx = base + f;
+            const int t = (idx / G) * C::RS + rg;
+            s_buf[t * G + idx % G] = t < n_valid ? part[f] : -CUDART_INF_F;
+        }
+        __syncwarp();
+
+        // ---- online softmax for head lane % G over this block
+        float sv[C::ENT];
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int e = 0; e < C::ENT; ++e) {
+            const int idx = lane + 32 * e;
+            sv[e] = idx < kBlockSize * G ? s_buf[idx] : -CUDART_INF_F;
+            mx = fmaxf(mx, sv[e]);
+        }
+#pragma unroll
+        for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m_own, mx);
+        float alpha = 1.f, psum = 0.f;
+        if (m_new != -CUDART_INF_F) {
+            alpha = exp2f(m_own - m_new);
+#pragma unroll
+            for (int e = 0; e < C::ENT; ++e) {
+                sv[e] = exp2f(sv[e] - m_new);
+                psum += sv[e];
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < C::ENT; ++e) sv[e] = 0.f;
+        }
+        l_own = l_own * alpha + psum;
+        m_own = m_new;
+#pragma unroll
+        for (int e = 0; e < C::ENT; ++e) {
+            const int idx = lane + 32 * e;
+            if (idx < kBlockSize * G) s_buf[idx] = sv[e];
+        }
+        __syncwarp();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float a = __shfl_sync(0xffffffffu, alpha, g);
+#pragma unroll
+                for (int e = 0; e < C::EPL; ++e) acc[g][e] *= a;
+            }
+        }
+
+        // ---- O += P . V
+#pragma unroll
+        for (int st = 0; st < C::STEPS; ++st) {
+            const int t = st * C::RS + rg;
+            float pr[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) pr[g] = s_buf[t * G + g];
+            float vf[C::EPL];
+#pragma unroll
+            for (int ch = 0; ch < C::CH; ++ch) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(vb + t * C::R + (ch * C::L + j) * 16);
+                Widen<T>::apply(raw, &vf[ch * C::VE]);
+            }
+            if (t < n_valid) {
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < C::EPL; e += 2)
+                        ffma2(acc[g][e], acc[g][e + 1], pr[g], pr[g], vf[e], vf[e + 1]);
+            }
+        }
+        __syncwarp();
+        if (issued < nb_w) issue(issued++);
+    }
+    if (failed) {
+        // Let copies still in flight land before the ring is reused.
+        for (int kk = k; kk < issued; ++kk) mbar_wait(bars + 8 * (kk % C::NSTAGE), (kk / C::NSTAGE) & 1);
+    }
+
+    // ---- merge the warps (and each warp's row groups) of this CTA
+#pragma unroll
+    for (int off = G; off < 32; off <<= 1) l_own += __shfl_xor_sync(0xffffffffu, l_own, off);
+    __syncthreads();
+    float *red_acc = reinterpret_cast<float *>(smem);  // [warp][rg][g][D]
+    float *red_m = reinterpret_cast<float *>(smem + C::OFF_ML);
+    float *red_l = red_m + kDecodeWarps * G;
+    if (lane < G) {
+        red_m[warp * G + lane] = m_own;
+        red_l[warp * G + lane] = l_own;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int ch = 0; ch < C::CH; ++ch) {
+            float *dst = red_acc + ((warp * C::RS + rg) * G + g) * D + (ch * C::L + j) * C::VE;
+#pragma unroll
+            for (int e = 0; e < C::VE; e += 4)
+                *reinterpret_cast<float4 *>(dst + e) =
+                    make_float4(acc[g][ch * C::VE + e], acc[g][ch * C::VE + e + 1], acc[g][ch * C::VE + e + 2],
+                                acc[g][ch * C::VE + e + 3]);
+        }
+    __syncthreads();
+
+    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
+        const int g = idx / D, d = idx % D;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, red_m[w * G + g]);
+        float O = 0.f, Lsum = 0.f;
+        if (M != -CUDART_INF_F) {
+#pragma unroll
+            for (int w = 0; w < kDecodeWarps; ++w) {
+                const float mw = red_m[w * G + g];
+                if (mw == -CUDART_INF_F) continue;
+                const float wt = exp2f(mw - M);
+                float o = 0.f;
+#pragma unroll
+                for (int r = 0; r < C::RS; ++r) o += red_acc[((w * C::RS + r) * G + g) * D + d];
+                O += wt * o;
+                Lsum += wt * red_l[w * G + g];
+            }
+        }
+        const int h = hk * G + g;
+        if (parts == 1) {
+            T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
+            store_out(out, Lsum > 0.f ? O / Lsum : 0.f);
+        } else {
+            const size_t pi = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts + p;
+            prm.ws_o[pi * D + d] = O;
+            if (d == 0) {
+                prm.ws_m[pi] = M;
+                prm.ws_l[pi] = Lsum;
+            }
+        }
+    }
+}
+
+// Merge the partitions of every sequence that has more than one:
+//   M = max_p m_p,  L = sum_p 2^(m_p - M) l_p,  out = sum_p 2^(m_p - M) O_p / L.
+// Grid (H, B), one thread per output element of a head.
+template <typename T>
+__global__ void decode_reduce_kernel(const DecodeParams prm, int D) {
+    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+    const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
+    const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
+    const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
+    if (parts == 1) return;
+    const size_t base = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts;
+    float M = -CUDART_INF_F;
+    for (int p = 0; p < parts; ++p) M = fmaxf(M, prm.ws_m[base + p]);
+    float O = 0.f, L = 0.f;
+    for (int p = 0; p < parts; ++p) {
+        const float mp = prm.ws_m[base + p];
+        if (mp == -CUDART_INF_F) continue;
+        const float wt = exp2f(mp - M);
+        L += wt * prm.ws_l[base + p];
+        O += wt * prm.ws_o[(base + p) * D + d];
+    }
+    T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
+    store_out(out, L > 0.f ? O / L : 0.f);
+}
+
+}  // namespace pa

@@ -1,0 +1,279 @@
+// libpa.so: the C ABI declared in include/pa.h.
+//
+// Host side only: argument checks, launch geometry and template dispatch.
+// Every step of the computation runs in the kernels this file includes.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <atomic>
+
+#include "pa_common.cuh"
+#include "decode.cuh"
+#include "prefill_sm100.cuh"
+#include "reshape_and_cache.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    int n = __atomic_load_n(&g_sm_count[dev], __ATOMIC_ACQUIRE);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        __atomic_store_n(&g_sm_count[dev], n, __ATOMIC_RELEASE);
+    }
+    return n;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = static_cast<int>(e);
+    return PA_ERR_CUDA;
+}
+
+int check_launch() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PA_OK : cuda_fail(e);
+}
+
+int check_shape(const pa_shape *s) {
+    if (!s) return PA_ERR_INVALID_ARGUMENT;
+    if (s->num_heads <= 0 || s->num_kv_heads <= 0 || s->num_blocks <= 0) return PA_ERR_INVALID_ARGUMENT;
+    if (s->num_heads % s->num_kv_heads != 0) return PA_ERR_INVALID_ARGUMENT;
+    if (s->block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    if (s->head_dim != 64 && s->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (s->dtype != PA_DTYPE_F32 && s->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+    const int g = s->num_heads / s->num_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return PA_ERR_UNSUPPORTED;
+    if (s->num_blocks > (int64_t{1} << 31) / PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;  // slots fit in int32 math
+    return PA_OK;
+}
+
+int elem_bytes(const pa_shape *s) { return s->dtype == PA_DTYPE_BF16 ? 2 : 4; }
+
+// Tokens per split-context partition. A context of at most one partition is
+// handled by the single pass alone (no workspace, no reduce kernel).
+int partition_tokens(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s) {
+    if (requested > 0) return requested;
+    const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    int tp = 512;
+    // small batches: shorter partitions so the grid still covers the GPU
+    while (tp > 128 && units * ((max_context_len + tp - 1) / tp) < 2 * sms) tp /= 2;
+    if (max_context_len <= tp) {
+        const int whole = ((max_context_len + 63) / 64) * 64;
+        return whole < 64 ? 64 : whole;
+    }
+    return tp;
+}
+
+struct DecodeGeometry {
+    int part_tokens;
+    int max_parts;
+    int64_t ws_bytes;
+};
+
+int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s,
+                    DecodeGeometry *g) {
+    if (num_seqs < 0 || max_context_len < 0) return PA_ERR_INVALID_ARGUMENT;
+    if (requested < 0 || (requested > 0 && (requested % 64 != 0))) return PA_ERR_INVALID_ARGUMENT;
+    g->part_tokens = partition_tokens(num_seqs, max_context_len, requested, s);
+    g->max_parts = max_context_len > 0 ? (max_context_len + g->part_tokens - 1) / g->part_tokens : 1;
+    if (g->max_parts < 1) g->max_parts = 1;
+    if (g->max_parts == 1) {
+        g->ws_bytes = 0;
+    } else {
+        const int64_t n = static_cast<int64_t>(num_seqs) * s->num_heads * g->max_parts;
+        const int64_t o_bytes = n * s->head_dim * 4;
+        g->ws_bytes = o_bytes + ((n * 4 + 15) / 16) * 16 * 2;
+    }
+    return PA_OK;
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory, once per device.
+template <typename K>
+int allow_smem(K kernel, int bytes, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const uint64_t bit = uint64_t{1} << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return PA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return PA_OK;
+}
+
+template <typename T, int D, int G>
+int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
+    using C = pa::DecodeCfg<T, D, G>;
+    static std::atomic<uint64_t> smem_done{0};
+    int arc = allow_smem(pa::decode_kernel<T, D, G>, C::SMEM, smem_done);
+    if (arc != PA_OK) return arc;
+    const dim3 grid(prm.max_parts, prm.num_kv_heads, num_seqs);
+    pa::decode_kernel<T, D, G><<<grid, pa::kDecodeThreads, C::SMEM, st>>>(prm);
+    int rc = check_launch();
+    if (rc != PA_OK || prm.max_parts == 1) return rc;
+    const dim3 rgrid(prm.num_heads, num_seqs);
+    pa::decode_reduce_kernel<T><<<rgrid, D, 0, st>>>(prm, D);
+    return check_launch();
+}
+
+template <typename T, int D>
+int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
+    switch (g) {
+        case 1: return launch_decode<T, D, 1>(prm, num_seqs, st);
+        case 2: return launch_decode<T, D, 2>(prm, num_seqs, st);
+        case 4: return launch_decode<T, D, 4>(prm, num_seqs, st);
+        case 8: return launch_decode<T, D, 8>(prm, num_seqs, st);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_abi_version(void) { return PA_ABI_VERSION; }
+
+const char *pa_strerror(int code) {
+    switch (code) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case PA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case PA_ERR_WORKSPACE: return "workspace missing or too small";
+        case PA_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+        case PA_ERR_DEVICE: return "no usable sm_100 device";
+        default: return "unknown error";
+    }
+}
+
+int pa_last_cuda_error(void) { return g_last_cuda_error; }
+
+int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                         int64_t num_tokens, const pa_shape *shape, void *stream) {
+    int rc = check_shape(shape);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARGUMENT;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(slot_mapping, 8))
+        return PA_ERR_ALIGNMENT;
+    const int row_bytes = shape->num_kv_heads * shape->head_dim * elem_bytes(shape);
+    if (row_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+    const int row_vecs = row_bytes / 16;
+    const int64_t total = num_tokens * row_vecs;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    if (blocks > int64_t{sms} * 16) blocks = int64_t{sms} * 16;
+    pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
+        static_cast<uint4 *>(v_cache), slot_mapping, num_tokens, shape->num_blocks * PA_BLOCK_SIZE, row_vecs);
+    return check_launch();
+}
+
+int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int32_t partition_tokens,
+                                  const pa_shape *shape) {
+    int rc = check_shape(shape);
+    if (rc != PA_OK) return rc;
+    DecodeGeometry g;
+    rc = decode_geometry(num_seqs, max_context_len, partition_tokens, shape, &g);
+    if (rc != PA_OK) return rc;
+    return g.ws_bytes;
+}
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+              float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes, const pa_shape *shape,
+              void *stream) {
+    int rc = check_shape(shape);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARGUMENT;
+    if (max_blocks_per_seq < 1 || !std::isfinite(scale)) return PA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_tables, 4) ||
+        !aligned(context_lens, 4))
+        return PA_ERR_ALIGNMENT;
+    DecodeGeometry g;
+    rc = decode_geometry(num_seqs, max_context_len, partition_tokens, shape, &g);
+    if (rc != PA_OK) return rc;
+    if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;  // grid z / y limit
+    pa::DecodeParams prm{};
+    if (g.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < g.ws_bytes) return PA_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return PA_ERR_ALIGNMENT;
+        const int64_t n = static_cast<int64_t>(num_seqs) * shape->num_heads * g.max_parts;
+        char *w = static_cast<char *>(workspace);
+        prm.ws_o = reinterpret_cast<float *>(w);
+        prm.ws_m = reinterpret_cast<float *>(w + n * shape->head_dim * 4);
+        prm.ws_l = reinterpret_cast<float *>(w + n * shape->head_dim * 4 + ((n * 4 + 15) / 16) * 16);
+    }
+    prm.out = out;
+    prm.q = q;
+    prm.k_cache = k_cache;
+    prm.v_cache = v_cache;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.num_blocks = shape->num_blocks;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_heads = shape->num_heads;
+    prm.num_kv_heads = shape->num_kv_heads;
+    prm.max_context_len = max_context_len;
+    prm.part_tokens = g.part_tokens;
+    prm.max_parts = g.max_parts;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    const int G = shape->num_heads / shape->num_kv_heads;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (shape->dtype == PA_DTYPE_BF16) {
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, 128>(G, prm, num_seqs, st)
+                                      : dispatch_g<__nv_bfloat16, 64>(G, prm, num_seqs, st);
+    }
+    return shape->head_dim == 128 ? dispatch_g<float, 128>(G, prm, num_seqs, st)
+                                  : dispatch_g<float, 64>(G, prm, num_seqs, st);
+}
+
+int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                     int32_t max_blocks_per_seq, const int32_t *cu_q_lens, const int32_t *context_lens,
+                     int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens, float scale, const pa_shape *shape,
+                     void *stream) {
+    int rc = check_shape(shape);
+    if (rc != PA_OK) return rc;
+    if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || max_q_len < 0 || num_q_tokens < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
+    if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens)
+        return PA_ERR_INVALID_ARGUMENT;
+    if (max_blocks_per_seq < 1 || !std::isfinite(scale)) return PA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_tables, 4) ||
+        !aligned(cu_q_lens, 4) || !aligned(context_lens, 4))
+        return PA_ERR_ALIGNMENT;
+    return pa::launch_prefill(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, cu_q_lens, context_lens,
+                              num_seqs, max_q_len, num_q_tokens, scale, shape, static_cast<cudaStream_t>(stream));
+}
+
+int pa_get_status(uint32_t *status, void *stream) {
+    if (!status) return PA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, pa::g_status, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(pa::g_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *status = v;
+    return PA_OK;
+}
+
+}  // extern "C"

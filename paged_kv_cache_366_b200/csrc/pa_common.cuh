@@ -1,0 +1,167 @@
+// Device helpers shared by the paged-attention kernels (sm_100a only).
+//
+// Hand-written PTX for the asynchronous-copy machinery: mbarriers, 1-D bulk
+// copies from global to shared memory, and the packed two-wide fp32 FMA.
+// Every wait here has a time limit. A wait that runs out sets a flag in the
+// library's device status word and returns false, so a kernel can never spin
+// forever.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+// Device status word of this library (PA_STATUS_* flags); read by pa_get_status.
+// The library is a single translation unit, so this is its one definition.
+__device__ unsigned int g_status = 0;
+
+constexpr int kBlockSize = PA_BLOCK_SIZE;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s for any single wait
+
+__device__ __forceinline__ void flag_status(unsigned int f) { atomicOr(&g_status, f); }
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---- mbarrier ---------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier to complete, for at most kWaitLimitNs.
+// Returns false (and flags PA_STATUS_WAIT_TIMEOUT) if it did not.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            flag_status(PA_STATUS_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// ---- bulk async copy (TMA, non-tensor) ---------------------------------------
+
+// Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory; completion is counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (createpolicy result).
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ---- arithmetic ---------------------------------------------------------------
+
+// (d0, d1) += (a0, a1) * (b0, b1), each lane an IEEE fma with round-to-nearest.
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rd, {%0, %1};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Widen 16 bytes of storage to fp32: 8 bf16 or 4 fp32 values.
+template <typename T>
+struct Widen;
+
+template <>
+struct Widen<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void apply(const uint4 &r, float *f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+template <>
+struct Widen<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void apply(const uint4 &r, float *f) {
+        f[0] = __uint_as_float(r.x);
+        f[1] = __uint_as_float(r.y);
+        f[2] = __uint_as_float(r.z);
+        f[3] = __uint_as_float(r.w);
+    }
+};
+
+__device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float load_in(const float *p) { return *p; }
+__device__ __forceinline__ float load_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+// Context length as the kernels use it: negative lengths count as 0 and
+// lengths over the table's capacity or the host's bound are clamped; both
+// set PA_STATUS_BAD_CONTEXT (only `report` callers flag, to flag once).
+__device__ __forceinline__ int clamp_context(int c, int cap, bool report) {
+    if (c < 0 || c > cap) {
+        if (report) flag_status(PA_STATUS_BAD_CONTEXT);
+        c = c < 0 ? 0 : cap;
+    }
+    return c;
+}
+
+}  // namespace pa

@@ -1,0 +1,200 @@
+"""Python binding of libpa.so: the C ABI in include/pa.h, same names.
+
+Argument marshalling only. Each call checks that its tensors are CUDA,
+contiguous and of the expected dtype, passes their pointers and the current
+torch stream to the C entry point, and raises PaError on a nonzero return.
+Every step of the computation runs in the library's kernels. There is no
+fallback: if libpa.so is missing, importing this module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
+BLOCK_SIZE = 16
+
+PA_STATUS_BAD_BLOCK_ID = 0x1
+PA_STATUS_BAD_SLOT = 0x2
+PA_STATUS_BAD_CONTEXT = 0x4
+PA_STATUS_WAIT_TIMEOUT = 0x8
+PA_STATUS_BAD_QUERY = 0x10
+
+
+class PaShape(ctypes.Structure):
+    _fields_ = [
+        ("num_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int64),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+EXPORTED = [
+    "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
+    "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version",
+]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libpa.so not built at %s: run paged_kv_cache_366_b200/build.py" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    SP = ctypes.POINTER(PaShape)
+    lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I64, SP, P]
+    lib.pa_reshape_and_cache.restype = ctypes.c_int
+    lib.pa_decode_workspace_bytes.argtypes = [I32, I32, I32, SP]
+    lib.pa_decode_workspace_bytes.restype = I64
+    lib.pa_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
+    lib.pa_decode.restype = ctypes.c_int
+    lib.pa_prefill_chunk.argtypes = [P, P, P, P, P, I32, P, P, I32, I32, I32, F, SP, P]
+    lib.pa_prefill_chunk.restype = ctypes.c_int
+    lib.pa_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+    lib.pa_get_status.restype = ctypes.c_int
+    lib.pa_strerror.argtypes = [ctypes.c_int]
+    lib.pa_strerror.restype = ctypes.c_char_p
+    lib.pa_last_cuda_error.argtypes = []
+    lib.pa_last_cuda_error.restype = ctypes.c_int
+    lib.pa_abi_version.argtypes = []
+    lib.pa_abi_version.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+class PaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        msg = "%s: %s (%d)" % (fn, lib.pa_strerror(code).decode(), code)
+        if code == -5:
+            msg += ", cudaError %d" % lib.pa_last_cuda_error()
+        super().__init__(msg)
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise PaError(fn, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return PA_DTYPE_BF16
+    if dt == torch.float32:
+        return PA_DTYPE_F32
+    raise ValueError("dtype must be bfloat16 or float32, got %s" % dt)
+
+
+def shape_of(k_cache: torch.Tensor, num_heads: int) -> PaShape:
+    """pa_shape of a pool [NB, 16, Hk, D] read by `num_heads` query heads."""
+    if k_cache.dim() != 4:
+        raise ValueError("k_cache must be [num_blocks, block_size, num_kv_heads, head_dim]")
+    nb, bs, hk, d = k_cache.shape
+    return PaShape(num_heads=int(num_heads), num_kv_heads=int(hk), head_dim=int(d), block_size=int(bs),
+                   num_blocks=int(nb), dtype=_dtype_code(k_cache.dtype))
+
+
+def _same_dtype(*ts):
+    dts = {t.dtype for t in ts}
+    if len(dts) != 1:
+        raise ValueError("q/k/v/caches/out must share one dtype, got %s" % sorted(map(str, dts)))
+
+
+def _int(t: torch.Tensor, dt: torch.dtype, name: str):
+    if t.dtype != dt:
+        raise ValueError("%s must be %s" % (name, dt))
+
+
+def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """Write each new token's K/V row into its slot of the pool (bit-exact copy)."""
+    _same_dtype(k, v, k_cache, v_cache)
+    _int(slot_mapping, torch.int64, "slot_mapping")
+    shape = shape_of(k_cache, k_cache.shape[2])
+    if k.shape[1:] != k_cache.shape[2:] or v.shape != k.shape or slot_mapping.shape[0] != k.shape[0]:
+        raise ValueError("k, v must be [T, Hk, D] matching the cache; slot_mapping [T]")
+    _check("pa_reshape_and_cache",
+           lib.pa_reshape_and_cache(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                    k.shape[0], ctypes.byref(shape), _stream(stream)))
+
+
+def pa_decode_workspace_bytes(num_seqs: int, max_context_len: int, partition_tokens: int, shape: PaShape) -> int:
+    n = lib.pa_decode_workspace_bytes(int(num_seqs), int(max_context_len), int(partition_tokens),
+                                      ctypes.byref(shape))
+    if n < 0:
+        raise PaError("pa_decode_workspace_bytes", int(n))
+    return int(n)
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+              partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Decode attention of one query token per sequence over its paged context."""
+    _same_dtype(out, q, k_cache, v_cache)
+    _int(block_tables, torch.int32, "block_tables")
+    _int(context_lens, torch.int32, "context_lens")
+    B, H, D = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
+    shape = shape_of(k_cache, H)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode",
+           lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                         block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
+                         int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape), _stream(stream)))
+
+
+def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
+                     scale: float, stream=None) -> None:
+    """Causal attention of query chunks at their context offsets (bf16, D=128)."""
+    _same_dtype(out, q, k_cache, v_cache)
+    _int(block_tables, torch.int32, "block_tables")
+    _int(cu_q_lens, torch.int32, "cu_q_lens")
+    _int(context_lens, torch.int32, "context_lens")
+    T, H, D = q.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or block_tables.shape[0] != B or cu_q_lens.shape[0] != B + 1:
+        raise ValueError("q, out [T, H, D]; block_tables [B, MB]; cu_q_lens [B+1]; context_lens [B]")
+    shape = shape_of(k_cache, H)
+    _check("pa_prefill_chunk",
+           lib.pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                block_tables.shape[1], _ptr(cu_q_lens), _ptr(context_lens), B, int(max_q_len), T,
+                                float(scale), ctypes.byref(shape), _stream(stream)))
+
+
+def pa_get_status(stream=None) -> int:
+    """Synchronize the stream, return and clear the device status word (PA_STATUS_* flags)."""
+    v = ctypes.c_uint32(0)
+    _check("pa_get_status", lib.pa_get_status(ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def pa_strerror(code: int) -> str:
+    return lib.pa_strerror(int(code)).decode()
+
+
+def pa_abi_version() -> int:
+    return int(lib.pa_abi_version())

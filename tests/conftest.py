@@ -8,3 +8,12 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_sessionstart(session):
+    # Both native libraries are built in-tree; rebuild them if a source is newer.
+    import oracle
+    from paged_kv_cache_366_b200 import build
+
+    oracle.build()
+    build.build()
