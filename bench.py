@@ -1,0 +1,539 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged-KV attention hot path on B200.
+
+One step is the whole path for one batch: the KV write of this step's new
+tokens (pa_reshape_and_cache), then paged decode over every decode sequence
+(pa_decode: the split-context kernel, plus the merge kernel when a context
+spans several partitions). The mixed workload also runs the causal prefill
+chunk (pa_prefill_chunk). Inputs are synthetic, seeded and resident in HBM
+before the timed region. Each step is captured once as CUDA graphs and
+replayed between CUDA events on the launching stream. A 256 MiB memset
+flushes L2 before every step, outside the events.
+
+Output: one JSON line on rank 0. `value` is the step's algorithmic bytes
+over the step time, in GB/s and summed over ranks (N > 1 runs independent
+replicas, with no data exchange). `roofline` rates the decode call (its
+algorithmic bytes over its event time) against the measured HBM copy
+bandwidth. `e2e` times the public DecodeStep API from pinned host buffers,
+with the copies inside. `cpu_baseline` is the fp64 oracle on the host cores.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_366_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; decode tokens/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
+WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "tiny"]
+
+
+# ---------------------------------------------------------------------------
+# Workload bookkeeping (host side)
+
+def split_seqs(case):
+    """Decode sequences (one new token) and prefill sequences (a chunk), each a contiguous range."""
+    ql = case.q_lens
+    dec = np.nonzero(ql == 1)[0]
+    pre = np.nonzero(ql > 1)[0]
+    for r in (dec, pre):
+        if len(r):
+            assert np.array_equal(r, np.arange(r[0], r[-1] + 1)), "decode/prefill sequences must be contiguous"
+    return dec, pre
+
+
+def step_bytes(case, dec, pre):
+    """Algorithmic bytes of one step, by part."""
+    E, H, Hk, D = case.elem_bytes, case.num_heads, case.num_kv_heads, case.head_dim
+    ctx = case.context_lens.astype(np.int64)
+    T = case.num_tokens
+    write = T * Hk * D * E * 2 * 2 + T * 8
+    kv_dec = int(ctx[dec].sum()) * Hk * D * E * 2
+    tables_dec = int(((ctx[dec] + 15) // 16).sum()) * 4 + 4 * len(dec)
+    decode = kv_dec + len(dec) * H * D * E * 2 + tables_dec
+    prefill = 0
+    if len(pre):
+        qt = int(case.q_lens[pre].sum())
+        prefill = int(ctx[pre].sum()) * Hk * D * E * 2 + qt * H * D * E * 2 + int(((ctx[pre] + 15) // 16).sum()) * 4
+    return {"write": write, "decode": decode, "kv_decode": kv_dec, "prefill": prefill,
+            "total": write + decode + prefill}
+
+
+def prefill_flops(case, pre):
+    H, D = case.num_heads, case.head_dim
+    f = 0
+    for b in pre:
+        c, q = int(case.context_lens[b]), int(case.q_lens[b])
+        o = c - q
+        f += sum((o + j + 1) for j in range(q)) * H * D * 4
+    return f
+
+
+def describe(case, dec, pre):
+    ctx = case.context_lens
+    d = {"workload": case.name, "num_seqs": int(case.num_seqs), "num_heads": case.num_heads,
+         "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim, "block_size": case.block_size,
+         "kv_dtype": case.dtype, "pool_blocks": int(case.num_blocks), "seed": case.seed,
+         "decode_seqs": int(len(dec)), "new_tokens": int(case.num_tokens),
+         "context_len_mean": float(ctx[dec].mean()) if len(dec) else 0.0,
+         "context_len_range": [int(ctx.min()), int(ctx.max())]}
+    if len(pre):
+        d["prefill_query_tokens"] = int(case.q_lens[pre].sum())
+    return d
+
+
+def load_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_sha():
+    h = hashlib.sha256()
+    for n in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_366_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """dram read+write bytes per decode launch from the committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_%s.md" % workload)
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.lstrip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+                    k, v = line.split(":", 1)
+                    kv[k.strip().strip("-* `")] = v.strip().strip("` ")
+        if kv.get("source_sha256") == decode_source_sha():
+            return float(kv["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, gpu: str):
+        self.samples = []
+        self.proc = None
+        q = ("timestamp,clocks.sm,clocks.max.sm,power.draw," +
+             ",".join("clocks_event_reasons." + r for r in REASONS))
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu, "--query-gpu=" + q,
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4 + len(REASONS):
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                self.samples.append((ts, float(parts[1]), float(parts[2]),
+                                     [r for r, v in zip(REASONS, parts[4:]) if v.lower() == "active"]))
+            except ValueError:
+                continue
+
+    def wait_ready(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
+    def summary(self, t0, t1):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if not self.samples:
+            return None
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # region shorter than the sampling period: nearest samples
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:2]
+        reasons = sorted({r for s in inside for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": max(s[2] for s in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+def gpu_id_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# Multi-rank plumbing (replicas: only timing and byte counts cross ranks)
+
+def aggregate(local_bytes: float, local_seconds: float):
+    """(sum of bytes over ranks, max of seconds over ranks); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return local_bytes, local_seconds
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    b = torch.tensor([local_bytes], dtype=torch.float64, device=dev)
+    t = torch.tensor([local_seconds], dtype=torch.float64, device=dev)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(b.item()), float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle: the cpu_baseline leg and the reference arm
+
+def oracle_step(case, seqs, num_threads):
+    """The oracle on the step for the listed decode sequences: cache write of their tokens, then decode."""
+    import oracle
+    rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in seqs], dtype=np.int64)
+    kc, vc = oracle.reshape_and_cache(case.k_new[rows], case.v_new[rows], case.k_cache, case.v_cache,
+                                      case.slot_mapping[rows])
+    oracle.decode(case.q[rows], kc, vc, case.block_tables[seqs], case.context_lens[seqs], case.scale,
+                  num_threads=num_threads)
+
+
+def step_bytes_for(case, seqs):
+    E, H, Hk, D = case.elem_bytes, case.num_heads, case.num_kv_heads, case.head_dim
+    ctx = case.context_lens[seqs].astype(np.int64)
+    n = len(seqs)
+    return (n * Hk * D * E * 4 + n * 8 + int(ctx.sum()) * Hk * D * E * 2 + n * H * D * E * 2 +
+            int(((ctx + 15) // 16).sum()) * 4 + 4 * n)
+
+
+def time_oracle(case, budget_s, min_reps=1):
+    """Oracle throughput on a bounded sample of the workload's decode sequences; returns a dict."""
+    dec, _ = split_seqs(case)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    t0 = time.perf_counter()
+    oracle_step(case, dec[:1], cores)
+    t_one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(len(dec), budget_s / t_one)))
+    seqs = dec[:n]
+    reps, spent = 0, 0.0
+    while reps < min_reps or spent < budget_s * 0.5:
+        t0 = time.perf_counter()
+        oracle_step(case, seqs, cores)
+        spent += time.perf_counter() - t0
+        reps += 1
+        if spent > budget_s:
+            break
+    nbytes = step_bytes_for(case, seqs) * reps
+    return {"value": nbytes / spent / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": "fp64 C oracle (OpenMP, %d threads): cache write + decode of the first %d of %d decode "
+                      "sequences of %s, %d repetition(s), %.2f s" % (cores, n, len(dec), case.name, reps, spent),
+            "seconds": spent}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    case = make_workload(args.workload)
+    dec, _ = split_seqs(case)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    # size each step's sample so warmup + steps fit in about two minutes
+    budget = max(0.005, 120.0 / (args.steps + args.warmup))
+    t0 = time.perf_counter()
+    oracle_step(case, dec[:1], cores)
+    t_one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(len(dec), budget / t_one)))
+    seqs = dec[:n]
+    for _ in range(args.warmup):
+        oracle_step(case, seqs, cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(case, seqs, cores)
+    dt = time.perf_counter() - t0
+    nbytes = step_bytes_for(case, seqs) * args.steps
+    value = nbytes / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": describe(case, dec, np.array([], np.int64)),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+                             "sample": "fp64 C oracle: each step = cache write + decode of the first %d of %d "
+                                       "decode sequences of %s" % (n, len(dec), case.name)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+
+def make_workload(name):
+    if name not in W.CONFIGS:
+        raise SystemExit("unknown workload %s (one of %s)" % (name, ", ".join(WORKLOADS)))
+    return W.CONFIGS[name]()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    from paged_kv_cache_366_b200 import pa
+    from paged_kv_cache_366_b200.step import DecodeStep
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+    case = make_workload(args.workload)
+    dec, pre = split_seqs(case)
+    nbytes = step_bytes(case, dec, pre)
+
+    k_cache, v_cache = dev(case.k_cache), dev(case.v_cache)
+    k_new, v_new, q = dev(case.k_new), dev(case.v_new), dev(case.q)
+    slots = dev(case.slot_mapping)
+    tables, lens, cu = dev(case.block_tables), dev(case.context_lens), dev(case.cu_q_lens)
+    shape = pa.shape_of(k_cache, case.num_heads)
+
+    d0, d1 = (int(dec[0]), int(dec[-1]) + 1) if len(dec) else (0, 0)
+    dec_rows = torch.from_numpy(np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)).cuda()
+    q_dec = q.index_select(0, dec_rows).contiguous() if len(dec) else None
+    out_dec = torch.empty_like(q_dec) if len(dec) else None
+    max_ctx = int(case.context_lens[dec].max()) if len(dec) else 0
+    ws_n = pa.pa_decode_workspace_bytes(len(dec), max_ctx, 0, shape) if len(dec) else 0
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
+    decode_kernels = 2 if ws_n else 1
+
+    if len(pre):
+        p0, p1 = int(pre[0]), int(pre[-1]) + 1
+        r0, r1 = int(case.cu_q_lens[p0]), int(case.cu_q_lens[p1])
+        q_pre = q[r0:r1].contiguous()
+        out_pre = torch.empty_like(q_pre)
+        cu_pre = (cu[p0:p1 + 1] - int(case.cu_q_lens[p0])).contiguous()
+        max_q = int(case.q_lens[pre].max())
+
+    stream = torch.cuda.Stream()
+
+    def do_write():
+        pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots)
+
+    def do_decode():
+        pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws)
+
+    def do_prefill():
+        pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
+                            case.scale)
+
+    parts = [("write", do_write)]
+    if len(pre):
+        parts.append(("prefill", do_prefill))
+    if len(dec):
+        parts.append(("decode", do_decode))
+    launches_per_step = 1 + (1 if len(pre) else 0) + (decode_kernels if len(dec) else 0)
+
+    graphs = []
+    with torch.cuda.stream(stream):
+        for _, fn in parts:  # eager once, then capture
+            fn()
+        stream.synchronize()
+        for _, fn in parts:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+    status = pa.pa_get_status(stream)
+    if status:
+        raise SystemExit("device status 0x%x after the first step" % status)
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    n_ev = len(parts) + 1
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            for g in graphs:
+                g.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_id_for(local_rank)) if rank == 0 else None
+    if sampler:
+        sampler.wait_ready()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            ev = events[i]
+            ev[0].record(stream)
+            for j, g in enumerate(graphs):
+                g.replay()
+                ev[j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall1 = time.time()
+    status = pa.pa_get_status(stream)
+    if status:
+        raise SystemExit("device status 0x%x after the timed steps" % status)
+
+    per_part = {name: 0.0 for name, _ in parts}
+    total = 0.0
+    for ev in events:
+        total += ev[0].elapsed_time(ev[-1]) * 1e-3
+        for j, (name, _) in enumerate(parts):
+            per_part[name] += ev[j].elapsed_time(ev[j + 1]) * 1e-3
+    sum_bytes, t_max = aggregate(float(nbytes["total"]) * args.steps, total)
+    value = sum_bytes / t_max / 1e9
+    ms_per_step = t_max / args.steps * 1e3
+
+    # end to end through the public API, host buffers, copies inside (decode workloads)
+    e2e = None
+    if len(dec) and not len(pre):
+        hk_cache = k_cache  # the pool is device-resident state
+        step = DecodeStep(hk_cache, v_cache, case.num_heads, len(dec), case.max_blocks_per_seq, max_ctx,
+                          case.scale)
+
+        def pinned(a):
+            t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16
+                                 else np.ascontiguousarray(a))
+            t = t.pin_memory()
+            return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
+        rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)
+        h_out = torch.empty(tuple(q_dec.shape), dtype=torch.int16 if case.dtype == "bf16" else torch.float32)
+        h_out = h_out.pin_memory()
+        if case.dtype == "bf16":
+            h_out = h_out.view(torch.bfloat16)
+        step.bind(pinned(case.q[rows]), pinned(case.k_new[rows]), pinned(case.v_new[rows]),
+                  pinned(case.slot_mapping[rows]), pinned(case.block_tables[d0:d1]),
+                  pinned(case.context_lens[d0:d1]), h_out)
+        n_e2e = max(10, min(args.steps, 500))
+        for _ in range(max(3, args.warmup)):
+            step.run()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+        barrier()
+        for i in range(n_e2e):
+            with torch.cuda.stream(step.stream):
+                flush.zero_()
+                ev[i][0].record(step.stream)
+            step.launch()
+            with torch.cuda.stream(step.stream):
+                ev[i][1].record(step.stream)
+            step.stream.synchronize()
+        barrier()
+        t_e2e = sum(a.elapsed_time(b) for a, b in ev) * 1e-3
+        b_e2e, t_e2e = aggregate(float(nbytes["total"]) * n_e2e, t_e2e)
+        e2e = {"value": b_e2e / t_e2e / 1e9, "unit": UNIT, "h2d_bytes_per_step": step.h2d_bytes(),
+               "d2h_bytes_per_step": step.d2h_bytes(), "steps": n_e2e,
+               "ms_per_step": t_e2e / n_e2e * 1e3, "api": "paged_kv_cache_366_b200.step.DecodeStep (CUDA graph)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    clocks = sampler.summary(wall0, wall1) if sampler else None
+    peak, peak_kind = load_peak()
+    roof = None
+    if len(dec):
+        t_dec = per_part["decode"] / args.steps
+        achieved = nbytes["decode"] / t_dec / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": profiled_traffic(args.workload), "kernel": "pa_decode (decode_kernel + merge)",
+                "algorithmic_bytes_per_launch": nbytes["decode"], "us_per_launch": t_dec * 1e6,
+                "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind}
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = time_oracle(case, args.cpu_seconds)
+        cpu.pop("seconds", None)
+    parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
+    config = describe(case, dec, pre)
+    config.update({"l2": "flushed before every step (256 MiB memset, outside the events)",
+                   "timing": "CUDA graph replay per part, CUDA events on the launching stream",
+                   "parallelism": "replicas" if args.gpus > 1 else "single GPU",
+                   "global_batch": int(case.num_seqs) * args.gpus})
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": case.dtype, "data": "synthetic (seeded; see paged_kv_cache_366_b200/"
+                                                                 "workloads.py)",
+            "config": config, "pct_of_hbm_peak": value / peak,
+            "decode_tokens_per_s": len(dec) * args.gpus / (t_max / args.steps),
+            "kv_gbs": nbytes["kv_decode"] * args.gpus / (t_max / args.steps) / 1e9,
+            "ms_per_part": parts_ms, "step_bytes": nbytes, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+            "wall_s_timed_region": wall1 - wall0}
+    if len(pre):
+        f = prefill_flops(case, pre)
+        t_pre = per_part["prefill"] / args.steps
+        line["prefill"] = {"flops": f, "us_per_launch": t_pre * 1e6, "tflops": f / t_pre / 1e12}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode_batch", choices=WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle timing")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -17,10 +17,10 @@
 //    loaded block from shared memory, so K/V cross HBM once per KV head.
 //  * The 4 warps of a CTA take the partition's blocks round-robin. Each warp
 //    streams its own blocks through an NSTAGE-deep shared-memory ring. A
-//    block's 16 K rows and 16 V rows are fetched by 32 TMA bulk copies (one
-//    per lane, a 256-byte row each at D=128 bf16) into a ring slot, and an
-//    mbarrier counts the bytes. Fetches run NSTAGE blocks ahead, so the
-//    table entry, the HBM fetch and the math of different blocks overlap.
+//    block's 16 K rows and 16 V rows of one KV head are two TMA tiled loads
+//    (a [16][D] box of the pool viewed as [NB*16][Hk][D]) into a ring slot,
+//    and an mbarrier counts the bytes. Fetches run NSTAGE blocks ahead, so
+//    the table entry, the HBM fetch and the math of different blocks overlap.
 //  * Lanes own column slices of a row made of CH 16-byte chunks (CH = 2, or 1
 //    for groups of 8 heads to bound registers), interleaved so shared-memory
 //    reads are conflict free. L = row_bytes / (16 * CH) lanes cover a row and RS = 32 / L rows are processed per step. q.k
@@ -35,6 +35,7 @@
 #include <math_constants.h>
 
 #include "pa_common.cuh"
+#include "tmap.cuh"
 
 namespace pa {
 
@@ -52,7 +53,12 @@ struct DecodeCfg {
     static constexpr int VE = 16 / E;                      // elements per 16-byte chunk
     static constexpr int EPL = CH * VE;                    // elements per lane per row
     static constexpr int STAGE_BYTES = 2 * kBlockSize * R; // K and V of one block
-    static constexpr int NSTAGE = STAGE_BYTES <= 8192 ? 3 : 2;
+    // Two stages per warp and three CTAs per SM (12 warps) measured faster on
+    // B200 than three stages at two CTAs per SM: more warps hide the math's
+    // latency better, and 12 x 2 x 8 KB in flight covers HBM latency.
+    static constexpr int NSTAGE = 2;
+    // CTAs per SM the register budget is sized for (wide rows keep more live state).
+    static constexpr int MIN_BLOCKS = G <= 4 ? 3 : 2;
     static constexpr int WARP_RING = NSTAGE * STAGE_BYTES;
     static constexpr int RING_BYTES = kDecodeWarps * WARP_RING;
     static constexpr int NPART = STEPS * G;                // q.k partials per lane per block
@@ -119,7 +125,9 @@ struct DecodeParams {
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams prm) {
+__global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS)
+    decode_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v) {
     using C = DecodeCfg<T, D, G>;
     const int p = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
@@ -154,8 +162,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq + blk0;
     int tbl = lane < nb_w ? __ldg(trow + warp + lane * kDecodeWarps) : 0;
     uint32_t bad_mask = 0;
-    const T *kc = static_cast<const T *>(prm.k_cache);
-    const T *vc = static_cast<const T *>(prm.v_cache);
 
     auto issue = [&](int k) {
         if (k >= 32 && (k & 31) == 0)
@@ -170,35 +176,37 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
             bad_mask &= ~(1u << s);
         }
         const uint32_t bar = bars + 8 * s;
-        if (lane == 0) mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-        __syncwarp();
-        const int row = lane & (kBlockSize - 1);
-        const T *src = (lane < kBlockSize ? kc : vc) +
-                       ((static_cast<size_t>(pb) * kBlockSize + row) * prm.num_kv_heads + hk) * D;
-        const uint32_t dst = ring_s + s * C::STAGE_BYTES + (lane < kBlockSize ? 0 : kBlockSize * C::R) + row * C::R;
-        bulk_g2s(dst, src, C::R, bar);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+            const uint32_t dst = ring_s + s * C::STAGE_BYTES;
+            tma_load_3d(dst, &tm_k, 0, hk, pb * kBlockSize, bar);
+            tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, hk, pb * kBlockSize, bar);
+        }
     };
 
-    // Queries of the group, pre-scaled by scale * log2(e).
-    float qf[G][C::EPL];
+    // Queries of the group, pre-scaled by scale * log2(e), as packed pairs.
+    constexpr int P2 = C::EPL / 2;  // packed pairs per lane per row
+    constexpr int VP = C::VE / 2;   // packed pairs per 16-byte chunk
+    f32x2 q2[G][P2];
     {
         const T *qb = static_cast<const T *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
+        const f32x2 sc = pack2(prm.scale_log2, prm.scale_log2);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + (ch * C::L + j) * C::VE));
-                Widen<T>::apply(raw, &qf[g][ch * C::VE]);
+                Widen<T>::apply2(raw, &q2[g][ch * VP]);
 #pragma unroll
-                for (int e = 0; e < C::VE; ++e) qf[g][ch * C::VE + e] *= prm.scale_log2;
+                for (int e = 0; e < VP; ++e) mul2(q2[g][ch * VP + e], sc);
             }
     }
 
-    float acc[G][C::EPL];
+    f32x2 acc2[G][P2];
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < C::EPL; ++e) acc[g][e] = 0.f;
+        for (int e = 0; e < P2; ++e) acc2[g][e] = 0ull;
     float m_own = -CUDART_INF_F;  // running max of head lane % G (log2 domain)
     float l_own = 0.f;            // this lane's share of that head's running sum
 
@@ -224,17 +232,19 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 #pragma unroll
         for (int st = 0; st < C::STEPS; ++st) {
             const int row = st * C::RS + rg;
-            float kf[C::EPL];
+            f32x2 k2[P2];
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(kb + row * C::R + (ch * C::L + j) * 16);
-                Widen<T>::apply(raw, &kf[ch * C::VE]);
+                Widen<T>::apply2(raw, &k2[ch * VP]);
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float a0 = 0.f, a1 = 0.f;
+                f32x2 s2 = 0ull;
 #pragma unroll
-                for (int e = 0; e < C::EPL; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1]);
+                for (int e = 0; e < P2; ++e) fma2(s2, q2[g][e], k2[e]);
+                float a0, a1;
+                unpack2(s2, a0, a1);
                 part[st * G + g] = a0 + a1;
             }
         }
@@ -284,8 +294,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const float a = __shfl_sync(0xffffffffu, alpha, g);
+                const f32x2 a2 = pack2(a, a);
 #pragma unroll
-                for (int e = 0; e < C::EPL; ++e) acc[g][e] *= a;
+                for (int e = 0; e < P2; ++e) mul2(acc2[g][e], a2);
             }
         }
 
@@ -296,18 +307,19 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
             float pr[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) pr[g] = s_buf[t * G + g];
-            float vf[C::EPL];
+            f32x2 v2[P2];
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(vb + t * C::R + (ch * C::L + j) * 16);
-                Widen<T>::apply(raw, &vf[ch * C::VE]);
+                Widen<T>::apply2(raw, &v2[ch * VP]);
             }
             if (t < n_valid) {
 #pragma unroll
-                for (int g = 0; g < G; ++g)
+                for (int g = 0; g < G; ++g) {
+                    const f32x2 p2 = pack2(pr[g], pr[g]);
 #pragma unroll
-                    for (int e = 0; e < C::EPL; e += 2)
-                        ffma2(acc[g][e], acc[g][e + 1], pr[g], pr[g], vf[e], vf[e + 1]);
+                    for (int e = 0; e < P2; ++e) fma2(acc2[g][e], p2, v2[e]);
+                }
             }
         }
         __syncwarp();
@@ -335,10 +347,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
         for (int ch = 0; ch < C::CH; ++ch) {
             float *dst = red_acc + ((warp * C::RS + rg) * G + g) * D + (ch * C::L + j) * C::VE;
 #pragma unroll
-            for (int e = 0; e < C::VE; e += 4)
-                *reinterpret_cast<float4 *>(dst + e) =
-                    make_float4(acc[g][ch * C::VE + e], acc[g][ch * C::VE + e + 1], acc[g][ch * C::VE + e + 2],
-                                acc[g][ch * C::VE + e + 3]);
+            for (int e = 0; e < VP; e += 2) {
+                float x0, x1, x2, x3;
+                unpack2(acc2[g][ch * VP + e], x0, x1);
+                unpack2(acc2[g][ch * VP + e + 1], x2, x3);
+                *reinterpret_cast<float4 *>(dst + 2 * e) = make_float4(x0, x1, x2, x3);
+            }
         }
     __syncthreads();
 

@@ -117,8 +117,15 @@ int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
     static std::atomic<uint64_t> smem_done{0};
     int arc = allow_smem(pa::decode_kernel<T, D, G>, C::SMEM, smem_done);
     if (arc != PA_OK) return arc;
+    CUtensorMap tm_k{}, tm_v{};
+    const uint64_t rows = static_cast<uint64_t>(prm.num_blocks) * pa::kBlockSize;
+    if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(T), D, 1, pa::kBlockSize,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(T), D, 1, pa::kBlockSize,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+        return PA_ERR_UNSUPPORTED;
     const dim3 grid(prm.max_parts, prm.num_kv_heads, num_seqs);
-    pa::decode_kernel<T, D, G><<<grid, pa::kDecodeThreads, C::SMEM, st>>>(prm);
+    pa::decode_kernel<T, D, G><<<grid, pa::kDecodeThreads, C::SMEM, st>>>(prm, tm_k, tm_v);
     int rc = check_launch();
     if (rc != PA_OK || prm.max_parts == 1) return rc;
     const dim3 rgrid(prm.num_heads, num_seqs);

@@ -107,17 +107,28 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 
 // ---- arithmetic ---------------------------------------------------------------
 
-// (d0, d1) += (a0, a1) * (b0, b1), each lane an IEEE fma with round-to-nearest.
-__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\t"
-        "mov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rd, {%0, %1};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
-        "mov.b64 {%0, %1}, rd;\n\t}"
-        : "+f"(d0), "+f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+// Packed pairs of fp32 in one 64-bit register, for the two-wide fp32 ops
+// (fma/mul .f32x2, sm_100). Each lane of a pair is an IEEE op with
+// round-to-nearest, so results equal two scalar ops.
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
 }
+
+__device__ __forceinline__ void unpack2(f32x2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// d += a * b
+__device__ __forceinline__ void fma2(f32x2 &d, f32x2 a, f32x2 b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+// d *= a
+__device__ __forceinline__ void mul2(f32x2 &d, f32x2 a) { asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a)); }
 
 // Widen 16 bytes of storage to fp32: 8 bf16 or 4 fp32 values.
 template <typename T>
@@ -126,6 +137,12 @@ struct Widen;
 template <>
 struct Widen<__nv_bfloat16> {
     static constexpr int N = 8;
+    // pairs (element 2i, element 2i+1) for i < 4
+    __device__ __forceinline__ static void apply2(const uint4 &r, f32x2 *f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+    }
     __device__ __forceinline__ static void apply(const uint4 &r, float *f) {
         const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
@@ -139,6 +156,10 @@ struct Widen<__nv_bfloat16> {
 template <>
 struct Widen<float> {
     static constexpr int N = 4;
+    __device__ __forceinline__ static void apply2(const uint4 &r, f32x2 *f) {
+        f[0] = (static_cast<f32x2>(r.y) << 32) | r.x;
+        f[1] = (static_cast<f32x2>(r.w) << 32) | r.z;
+    }
     __device__ __forceinline__ static void apply(const uint4 &r, float *f) {
         f[0] = __uint_as_float(r.x);
         f[1] = __uint_as_float(r.y);

@@ -44,10 +44,10 @@ EXPORTED = [
 ]
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError("libpa.so not built at %s: run paged_kv_cache_366_b200/build.py" % LIB_PATH)
-    lib = ctypes.CDLL(LIB_PATH)
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError("libpa.so not built at %s: run paged_kv_cache_366_b200/build.py" % path)
+    lib = ctypes.CDLL(path)
     P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     SP = ctypes.POINTER(PaShape)
     lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I64, SP, P]
