@@ -70,6 +70,7 @@ typedef enum {
     PA_ERR_WORKSPACE = -4,        /* workspace missing or smaller than pa_decode_workspace_bytes */
     PA_ERR_CUDA = -5,             /* a CUDA runtime call or launch failed */
     PA_ERR_DEVICE = -6,           /* no usable device, or not an sm_100 device */
+    PA_ERR_SCRATCH_LIMIT = -7,    /* pa_decode_noalloc: request larger than its built-in scratch */
 } pa_error;
 
 /* Flags of the device status word (OR-ed together). */
@@ -178,6 +179,42 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
                      const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *cu_q_lens,
                      const int32_t *context_lens, int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens,
                      float scale, const pa_shape *shape, void *stream);
+
+/*
+ * pa_decode_noalloc: pa_decode for callers that cannot allocate device memory.
+ * The paper has no counterpart to this call; it is a deployment convenience.
+ *
+ * Some callers have no way to get a scratch buffer. Examples: code that runs
+ * while a CUDA graph is being captured in a mode that forbids allocation; a
+ * host engine that has reserved nearly all of HBM for its own KV pool and owns
+ * every allocation; plugin code loaded into a runtime whose allocator it cannot
+ * reach; a latency-critical loop where cudaMalloc's implicit synchronization is
+ * not acceptable. This entry point computes exactly what pa_decode computes with
+ * the same arguments. It takes no workspace: the split-context partials go to a
+ * scratch array compiled into the library, PA_NOALLOC_SCRATCH_BYTES long.
+ *
+ *  - The array is a static device variable. Every GPU on which the library's
+ *    module is loaded holds those bytes until the process exits.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current, and caches it. Make that
+ *    first call outside any stream capture; later calls only enqueue kernels.
+ *  - Requests whose partials need more than PA_NOALLOC_SCRATCH_BYTES (see
+ *    pa_decode_workspace_bytes) return PA_ERR_SCRATCH_LIMIT and launch nothing.
+ *    Use pa_decode with your own workspace for those, or a larger
+ *    partition_tokens.
+ *  - Every call on a device shares the one array, and the array keeps whatever
+ *    the last call left in it. Nothing in it needs to start at zero: each call
+ *    writes every partial it later reads. Calls that may overlap on the GPU
+ *    (different streams, or different host threads on one device) race on the
+ *    array and must be serialized by the caller.
+ * The library calls no cudaMalloc, cudaFree or other allocating routine here.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                      int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                      const pa_shape *shape, void *stream);
 
 /*
  * pa_get_status: synchronize `stream`, copy the device status word of the

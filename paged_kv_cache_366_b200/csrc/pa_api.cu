@@ -159,6 +159,7 @@ const char *pa_strerror(int code) {
         case PA_ERR_WORKSPACE: return "workspace missing or too small";
         case PA_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
         case PA_ERR_DEVICE: return "no usable sm_100 device";
+        case PA_ERR_SCRATCH_LIMIT: return "request needs more scratch than pa_decode_noalloc's built-in array";
         default: return "unknown error";
     }
 }
@@ -266,6 +267,55 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
         return PA_ERR_ALIGNMENT;
     return pa::launch_prefill(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, cu_q_lens, context_lens,
                               num_seqs, max_q_len, num_q_tokens, scale, shape, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ---- pa_decode_noalloc: decode with a scratch array compiled into the library ----
+
+namespace {
+
+// Scratch for the split-context partials of pa_decode_noalloc. Each device
+// that loads this module holds it until the process exits. Host code must not
+// use the symbol itself as a device address: the address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+std::atomic<void *> g_noalloc_ptr[kMaxDevices];
+
+int noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_DEVICE;
+    void *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with `dev` current
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+    *ptr = p;
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                      int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                      const pa_shape *shape, void *stream) {
+    const int64_t need = pa_decode_workspace_bytes(num_seqs, max_context_len, partition_tokens, shape);
+    if (need < 0) return static_cast<int>(need);
+    if (need > static_cast<int64_t>(PA_NOALLOC_SCRATCH_BYTES)) return PA_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    if (need > 0) {
+        const int rc = noalloc_scratch(&scratch);
+        if (rc != PA_OK) return rc;
+    }
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                     max_context_len, scale, partition_tokens, scratch, need, shape, stream);
 }
 
 int pa_get_status(uint32_t *status, void *stream) {

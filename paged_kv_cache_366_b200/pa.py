@@ -40,8 +40,11 @@ class PaShape(ctypes.Structure):
 
 EXPORTED = [
     "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
-    "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version",
+    "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version", "pa_decode_noalloc",
 ]
+
+PA_ERR_SCRATCH_LIMIT = -7
+PA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def _load(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -58,6 +61,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode.restype = ctypes.c_int
     lib.pa_prefill_chunk.argtypes = [P, P, P, P, P, I32, P, P, I32, I32, I32, F, SP, P]
     lib.pa_prefill_chunk.restype = ctypes.c_int
+    lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, SP, P]
+    lib.pa_decode_noalloc.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_strerror.argtypes = [ctypes.c_int]
@@ -165,6 +170,29 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
            lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                          block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
                          int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape), _stream(stream)))
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+                      partition_tokens: int = 0, stream=None) -> None:
+    """pa_decode without a workspace argument, for callers that cannot allocate device memory.
+
+    The split-context partials go to a PA_NOALLOC_SCRATCH_BYTES array built
+    into the library (held on every device that loads it). Requests that need
+    more raise PaError with PA_ERR_SCRATCH_LIMIT. Calls that may overlap on
+    one GPU share that array and must not run concurrently. Make the first
+    call on each device outside stream capture.
+    """
+    _same_dtype(out, q, k_cache, v_cache)
+    _int(block_tables, torch.int32, "block_tables")
+    _int(context_lens, torch.int32, "context_lens")
+    B, H, D = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
+    shape = shape_of(k_cache, H)
+    _check("pa_decode_noalloc",
+           lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                 block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
+                                 int(partition_tokens), ctypes.byref(shape), _stream(stream)))
 
 
 def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
