@@ -52,7 +52,7 @@ int check_shape(const pa_shape *s) {
     if (s->dtype != PA_DTYPE_F32 && s->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
     const int g = s->num_heads / s->num_kv_heads;
     if (g != 1 && g != 2 && g != 4 && g != 8) return PA_ERR_UNSUPPORTED;
-    if (s->num_blocks > (int64_t{1} << 31) / PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;  // slots fit in int32 math
+    if (s->num_blocks >= (int64_t{1} << 31) / PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;  // rows fit in int32 math
     return PA_OK;
 }
 
