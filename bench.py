@@ -46,7 +46,7 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
-WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "tiny"]
+WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny"]
 
 
 # ---------------------------------------------------------------------------
@@ -103,12 +103,15 @@ def describe(case, dec, pre):
     return d
 
 
-def load_peak():
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def load_peak(key="hbm_gbs"):
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            return float(json.load(f)[key]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
 def decode_source_sha():
@@ -513,7 +516,15 @@ def run_ours(args):
     if len(pre):
         f = prefill_flops(case, pre)
         t_pre = per_part["prefill"] / args.steps
-        line["prefill"] = {"flops": f, "us_per_launch": t_pre * 1e6, "tflops": f / t_pre / 1e12}
+        tpeak, tkind = load_peak("bf16_tflops")
+        tf = f / t_pre / 1e12
+        line["prefill"] = {"flops": f, "us_per_launch": t_pre * 1e6, "tflops": tf,
+                           "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s",
+                                        "frac": tf / tpeak, "traffic": None,
+                                        "kernel": "prefill_kernel (tcgen05)",
+                                        "peak_kind": tkind + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}}
+        if not len(dec):
+            line["roofline"] = line["prefill"]["roofline"]
     print(json.dumps(line), flush=True)
     return 0
 

@@ -20,9 +20,11 @@
 //    M=128, N=128, K=16 per instruction) with accumulators in tensor memory:
 //    two S buffers and one O, 384 of the 512 columns. QK of tile j+1 is issued
 //    before the softmax of tile j, so the two overlap.
-//  * Softmax: thread r owns row r. It reads its S row from TMEM, masks keys past
-//    its causal limit, and keeps a running max in the exp2 domain. It writes P as
-//    bf16 into shared memory in the 128-byte-swizzled K-major layout the MMA
+//  * Softmax: 8 warps. The two warps that share a TMEM lane quarter split each
+//    row into 64-column halves and exchange partial maxima and sums through
+//    shared memory. They mask keys past the row's causal limit and keep a
+//    running max in the exp2 domain, with tree-shaped max/sum reductions. P goes
+//    as bf16 into shared memory in the 128-byte-swizzled K-major layout the MMA
 //    reads. O is rescaled in TMEM only when the row max grows by more than
 //    2^8; otherwise the older max is kept, and P stays below 256.
 //  * One thread issues the MMAs and commits them to mbarriers. Warp 0's lanes
@@ -130,7 +132,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 
 // ---- geometry -------------------------------------------------------------------
 
-constexpr int kPfThreads = 128;
+constexpr int kPfThreads = 256;
 constexpr int kPfM = 128;  // rows per CTA
 constexpr int kPfN = 128;  // keys per tile
 constexpr int kPfD = 128;  // head_dim
@@ -143,10 +145,11 @@ constexpr int kPfOffP = kPfOffV + 2 * kPfTile;
 constexpr int kPfOffBar = kPfOffP + kPfTile;    // mbarriers (8 B each)
 constexpr int kPfBars = 9;                      // q, k[2], v[2], s[2], o, spare
 constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;
-constexpr int kPfSmem = kPfOffSlot + 16 + 1024;  // + room to align the base to 1024 B
+constexpr int kPfOffRed = kPfOffSlot + 16;      // [2][128] floats: row max / row sum halves
+constexpr int kPfSmem = kPfOffRed + 2 * 128 * 4 + 1024;  // + room to align the base to 1024 B
 constexpr uint32_t kPfTmemCols = 512;
 constexpr int kPfBlocksPerTile = kPfN / kBlockSize;
-static_assert(kPfOffBar + kPfBars * 8 + 16 + 1024 <= 232448, "prefill shared memory over the 227 KB limit");
+static_assert(kPfSmem <= 232448, "prefill shared memory over the 227 KB limit");
 static_assert(kPfBlocksPerTile == 8, "warp 0 lanes 0..7 own one block each");
 
 struct PrefillParams {
@@ -221,8 +224,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS[2] = {tmem, tmem + 128};
-    const uint32_t tO = tmem + 256;
+    const uint32_t tO = tmem + 256;  // S tiles at columns 0 and 128
 
     // ---- loads (warp 0) ----
     const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq;
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kPfD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kPfHalf + (kk & 3) * 32;
-            umma_bf16(tS[t & 1], smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), kIdQK,
+            umma_bf16(tmem + (t & 1) * kPfN, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), kIdQK,
                       kk > 0);
         }
         umma_commit(bar_s + 8 * (t & 1));
@@ -304,13 +306,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
     }
 
-    // ---- per-row state (thread tid owns row tid) ----
-    const int r = tid;
+    // ---- per-row state: warps w and w+4 share TMEM lanes 32(w%4).., and each takes
+    // one 64-column half of the row (keys of the S tile, dims of O) ----
+    const int quarter = warp & 3, hcol = warp >> 2;
+    const int r = quarter * 32 + lane;
     const int tok = min(t0 + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
     const int pos = o + tok;                     // causal limit: keys 0..pos
     float m_ref = -CUDART_INF_F;                 // reference max (log2 domain) of the row
-    float l_sum = 0.f;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float l_sum = 0.f;                           // this thread's half of the row sum
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    float *red = reinterpret_cast<float *>(base + kPfOffRed);  // [2][128] partial row max, then sums
     int pv_issued = 0;
 
     for (int j = 0; j < n_tiles; ++j) {
@@ -335,7 +340,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (j > 0) {
             w = mbar_wait(bar_o, (j - 1) & 1) && w;
             tc_fence_after();
-            if (warp == 0 && j + 1 < n_tiles) load_tile(&tm_v, sV + ((j + 1) & 1) * kPfTile, bar_v + 8 * ((j + 1) & 1), row_a);
+            if (warp == 0 && j + 1 < n_tiles)
+                load_tile(&tm_v, sV + ((j + 1) & 1) * kPfTile, bar_v + 8 * ((j + 1) & 1), row_a);
         }
         if (warp == 0) {  // advance the table window: rows of tiles j+2, j+3, j+4
             row_a = row_b;
@@ -355,57 +361,70 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
         }
         __syncwarp();
-        // 4b. softmax of row r over tile j
-        float s[kPfN];
+        // 4b. this thread's 64 scores of row r
+        constexpr int HN = kPfN / 2;
+        float s[HN];
+        const uint32_t s_cols = tmem + (j & 1) * kPfN + hcol * HN;
 #pragma unroll
-        for (int ch = 0; ch < kPfN / 32; ++ch) {
+        for (int ch = 0; ch < HN / 32; ++ch) {
             float v[32];
-            tmem_ld32(tS[j & 1] + lane_base + ch * 32, v);
+            tmem_ld32(s_cols + lane_base + ch * 32, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[ch * 32 + i] = v[i] * prm.scale_log2;
         }
-        const int key0 = j * kPfN;
-        if (key0 + kPfN - 1 > pos) {
+        const int key0 = j * kPfN + hcol * HN;
+        if (key0 + HN - 1 > pos) {
 #pragma unroll
-            for (int i = 0; i < kPfN; ++i)
+            for (int i = 0; i < HN; ++i)
                 if (key0 + i > pos) s[i] = -CUDART_INF_F;
         }
-        float mx = -CUDART_INF_F;
+        float m8[8];
 #pragma unroll
-        for (int i = 0; i < kPfN; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int i = 8; i < HN; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
+        const float mx_half = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        red[hcol * kPfM + r] = mx_half;
+        __syncthreads();
+        const float mx = fmaxf(red[r], red[kPfM + r]);
         float alpha = 1.f;
         if (mx > m_ref + 8.f || m_ref == -CUDART_INF_F) {
             const float m_new = fmaxf(mx, m_ref);
             alpha = (m_ref == -CUDART_INF_F) ? 0.f : exp2f(m_ref - m_new);
             m_ref = m_new;
         }
-        float psum = 0.f;
-        unsigned char *prow = base + kPfOffP + r * 128;
+        float a8[8];
 #pragma unroll
-        for (int ch = 0; ch < kPfN / 8; ++ch) {
+        for (int i = 0; i < 8; ++i) a8[i] = 0.f;
+        unsigned char *prow = base + kPfOffP + hcol * kPfHalf + r * 128;
+#pragma unroll
+        for (int cc = 0; cc < HN / 8; ++cc) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float p0 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[ch * 8 + 2 * e] - m_ref);
-                const float p1 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[ch * 8 + 2 * e + 1] - m_ref);
+                const float p0 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[cc * 8 + 2 * e] - m_ref);
+                const float p1 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[cc * 8 + 2 * e + 1] - m_ref);
                 const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                psum += __low2float(pb) + __high2float(pb);
+                a8[(2 * e) & 7] += __low2float(pb);
+                a8[(2 * e + 1) & 7] += __high2float(pb);
                 pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
             }
-            const int half = ch >> 3, cc = ch & 7;
-            *reinterpret_cast<uint4 *>(prow + half * kPfHalf + ((cc ^ (r & 7)) << 4)) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+        const float psum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
         l_sum = l_sum * alpha + psum;
-        // rescale O rows in tensor memory (warp-uniform: tcgen05.ld/st are .sync.aligned)
+        // rescale this thread's half of O's row in tensor memory (warp-uniform:
+        // tcgen05.ld/st are .sync.aligned)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-            for (int ch = 0; ch < kPfD / 32; ++ch) {
+            for (int ch = 0; ch < HN / 32; ++ch) {
+                const uint32_t oc = tO + hcol * HN + lane_base + ch * 32;
                 float v[32];
-                tmem_ld32(tO + lane_base + ch * 32, v);
+                tmem_ld32(oc, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                tmem_st32(tO + lane_base + ch * 32, v);
+                tmem_st32(oc, v);
             }
         }
         // 5. P visible to the tensor core, TMEM reads/writes ordered before the next MMA
@@ -426,20 +445,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
 
-    // ---- epilogue: out = O / l for the valid rows ----
+    // ---- epilogue: out = O / l for the valid rows, each thread its 64 dims ----
     if (ok && pv_issued == n_tiles && n_tiles > 0) {
+        red[hcol * kPfM + r] = l_sum;
         ok = mbar_wait(bar_o, (n_tiles - 1) & 1);
+        ok = __syncthreads_and(ok ? 1 : 0) != 0;
         tc_fence_after();
         if (ok) {
+            const float l_row = red[r] + red[kPfM + r];
             const bool row_ok = r / G < rows_valid;
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
             const int orow = row_ok ? q0 + t0 + r / G : q0;
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
-                                 (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
+                                 (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD + hcol * 64;
 #pragma unroll
-            for (int ch = 0; ch < kPfD / 32; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 float v[32];
-                tmem_ld32(tO + lane_base + ch * 32, v);
+                tmem_ld32(tO + hcol * 64 + lane_base + ch * 32, v);
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
                     uint4 pkt;

@@ -327,10 +327,17 @@ def mixed_step(seed: int = 4, keep_logical: bool = False) -> PagedCase:
                      head_dim=128, dtype="bf16", keep_logical=keep_logical)
 
 
+def prefill_chunk(seed: int = 4, keep_logical: bool = False) -> PagedCase:
+    """The mixed step's prefill alone: one sequence, 2048 query tokens at offset 6144 (c = 8192)."""
+    return make_case("prefill_chunk", seed, context_lens=[8192], q_lens=[2048], num_heads=32, num_kv_heads=8,
+                     head_dim=128, dtype="bf16", keep_logical=keep_logical)
+
+
 CONFIGS = {
     "tiny": tiny,
     "decode_batch": decode_batch,
     "long_context": long_context,
     "prefix_sharing": prefix_sharing,
     "mixed_step": mixed_step,
+    "prefill_chunk": prefill_chunk,
 }
