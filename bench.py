@@ -7,8 +7,9 @@ tokens (pa_reshape_and_cache), then paged decode over every decode sequence
 spans several partitions). The mixed workload also runs the causal prefill
 chunk (pa_prefill_chunk). Inputs are synthetic, seeded and resident in HBM
 before the timed region. Each step is captured once as CUDA graphs and
-replayed between CUDA events on the launching stream. A 256 MiB memset
-flushes L2 before every step, outside the events.
+replayed between CUDA events on the launching stream. Before every step,
+outside the events, a 256 MiB memset and then a 256 MiB read flush L2 (the
+read makes the memset's dirty lines drain to HBM before the step starts).
 
 Output: one JSON line on rank 0. `value` is the step's algorithmic bytes
 over the step time, in GB/s and summed over ranks (N > 1 runs independent
@@ -382,6 +383,7 @@ def run_ours(args):
         parts.append(("decode", do_decode))
     launches_per_step = 1 + (1 if len(pre) else 0) + (decode_kernels if len(dec) else 0)
 
+    # one graph for the whole step (the headline), one per part (breakdown, roofline)
     graphs = []
     with torch.cuda.stream(stream):
         for _, fn in parts:  # eager once, then capture
@@ -392,29 +394,66 @@ def run_ours(args):
             with torch.cuda.graph(g, stream=stream):
                 fn()
             graphs.append(g)
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=stream):
+            for _, fn in parts:
+                fn()
     torch.cuda.synchronize()
     status = pa.pa_get_status(stream)
     if status:
         raise SystemExit("device status 0x%x after the first step" % status)
 
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    n_ev = len(parts) + 1
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    class _Flush:
+        """Evict L2: write a buffer larger than L2, then read another, so the write's
+        dirty lines reach HBM before the timed events rather than during them."""
+
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.sum(flush_r)
+
+    flush = _Flush()
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
+            flush.zero_()
+            g_step.replay()
             flush.zero_()
             for g in graphs:
                 g.replay()
     torch.cuda.synchronize()
 
+    # timed region: K steps, each one graph replay between events, L2 flushed before each
     sampler = ClockSampler(gpu_id_for(local_rank)) if rank == 0 else None
     if sampler:
         sampler.wait_ready()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
+            flush.zero_()
+            step_ev[i][0].record(stream)
+            g_step.replay()
+            step_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall1 = time.time()
+    status = pa.pa_get_status(stream)
+    if status:
+        raise SystemExit("device status 0x%x after the timed steps" % status)
+    total = sum(a.elapsed_time(b) for a, b in step_ev) * 1e-3
+
+    # per-part times (each part its own graph, events between), for the breakdown and rooflines
+    n_parts_steps = min(args.steps, 500)
+    n_ev = len(parts) + 1
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_parts_steps)]
+    with torch.cuda.stream(stream):
+        for i in range(n_parts_steps):
             flush.zero_()
             ev = events[i]
             ev[0].record(stream)
@@ -422,18 +461,11 @@ def run_ours(args):
                 g.replay()
                 ev[j + 1].record(stream)
     torch.cuda.synchronize()
-    barrier()
-    wall1 = time.time()
-    status = pa.pa_get_status(stream)
-    if status:
-        raise SystemExit("device status 0x%x after the timed steps" % status)
-
     per_part = {name: 0.0 for name, _ in parts}
-    total = 0.0
     for ev in events:
-        total += ev[0].elapsed_time(ev[-1]) * 1e-3
         for j, (name, _) in enumerate(parts):
             per_part[name] += ev[j].elapsed_time(ev[j + 1]) * 1e-3
+    per_part = {k: v * args.steps / n_parts_steps for k, v in per_part.items()}  # per-step sums as over K steps
     sum_bytes, t_max = aggregate(float(nbytes["total"]) * args.steps, total)
     value = sum_bytes / t_max / 1e9
     ms_per_step = t_max / args.steps * 1e3
@@ -499,8 +531,10 @@ def run_ours(args):
         cpu.pop("seconds", None)
     parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
-    config.update({"l2": "flushed before every step (256 MiB memset, outside the events)",
-                   "timing": "CUDA graph replay per part, CUDA events on the launching stream",
+    config.update({"l2": "flushed before every step, outside the events: 256 MiB memset, then a 256 MiB read "
+                         "so the memset's write-back is not charged to the step",
+                   "timing": "one CUDA graph replay per step between CUDA events on the launching stream; "
+                             "per-part times from a second loop of per-part graphs",
                    "parallelism": "replicas" if args.gpus > 1 else "single GPU",
                    "global_batch": int(case.num_seqs) * args.gpus})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,

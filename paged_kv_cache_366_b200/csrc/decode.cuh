@@ -9,7 +9,7 @@
 // and an accumulator O rescaled by exp(m_old - m_new) whenever m grows.
 //
 // How it runs on B200:
-//  * Grid (partition, KV head, sequence). A CTA owns one KV head of one
+//  * Grid (KV head, sequence, partition). A CTA owns one KV head of one
 //    sequence over one partition of the context (split-context pass).
 //    Sequences longer than a partition also write (m, l, O) partials, and
 //    decode_reduce_kernel merges them.
@@ -129,7 +129,13 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
     decode_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
     using C = DecodeCfg<T, D, G>;
-    const int p = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    // Grid (KV head, sequence, partition): every unit's first partition launches
+    // before any second one, so full partitions run first and the short last
+    // partitions (or empty CTAs) form the tail.
+    const int hk = blockIdx.x, b = blockIdx.y, p = blockIdx.z;
+    // Launched as a programmatic dependent (its launch overlaps the previous
+    // kernel, e.g. the cache write): wait for that kernel before reading any input.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
     const int c = clamp_context(__ldg(prm.context_lens + b), cap, p == 0 && hk == 0 && threadIdx.x == 0);
     const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
@@ -258,39 +264,28 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
         }
         __syncwarp();
 
-        // ---- online softmax for head lane % G over this block
+        // ---- online softmax for head lane % G over this block. The reference max
+        // m_own is updated (and O, l rescaled) only when a score exceeds it by more
+        // than 8 in the exp2 domain; otherwise the older max is kept and P stays
+        // below 2^8. The result is the same softmax, with fewer rescales.
         float sv[C::ENT];
-        float mx = -CUDART_INF_F;
+        bool grow = false;
 #pragma unroll
         for (int e = 0; e < C::ENT; ++e) {
             const int idx = lane + 32 * e;
             sv[e] = idx < kBlockSize * G ? s_buf[idx] : -CUDART_INF_F;
-            mx = fmaxf(mx, sv[e]);
+            grow |= sv[e] > m_own + 8.f;
         }
+        if (__any_sync(0xffffffffu, grow)) {
+            float mx = -CUDART_INF_F;
 #pragma unroll
-        for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m_own, mx);
-        float alpha = 1.f, psum = 0.f;
-        if (m_new != -CUDART_INF_F) {
-            alpha = exp2f(m_own - m_new);
+            for (int e = 0; e < C::ENT; ++e) mx = fmaxf(mx, sv[e]);
 #pragma unroll
-            for (int e = 0; e < C::ENT; ++e) {
-                sv[e] = exp2f(sv[e] - m_new);
-                psum += sv[e];
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < C::ENT; ++e) sv[e] = 0.f;
-        }
-        l_own = l_own * alpha + psum;
-        m_own = m_new;
-#pragma unroll
-        for (int e = 0; e < C::ENT; ++e) {
-            const int idx = lane + 32 * e;
-            if (idx < kBlockSize * G) s_buf[idx] = sv[e];
-        }
-        __syncwarp();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m_own, mx);
+            const float alpha = m_own == -CUDART_INF_F ? 0.f : exp2f(m_own - m_new);
+            l_own *= alpha;
+            m_own = m_new;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const float a = __shfl_sync(0xffffffffu, alpha, g);
@@ -299,6 +294,24 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
                 for (int e = 0; e < P2; ++e) mul2(acc2[g][e], a2);
             }
         }
+        float psum = 0.f;
+        if (m_own != -CUDART_INF_F) {
+#pragma unroll
+            for (int e = 0; e < C::ENT; ++e) {
+                sv[e] = exp2f(sv[e] - m_own);
+                psum += sv[e];
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < C::ENT; ++e) sv[e] = 0.f;
+        }
+        l_own += psum;
+#pragma unroll
+        for (int e = 0; e < C::ENT; ++e) {
+            const int idx = lane + 32 * e;
+            if (idx < kBlockSize * G) s_buf[idx] = sv[e];
+        }
+        __syncwarp();
 
         // ---- O += P . V
 #pragma unroll
@@ -388,28 +401,52 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
             }
         }
     }
+    // let the merge kernel (launched as a programmatic dependent) get scheduled
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the partitions of every sequence that has more than one:
 //   M = max_p m_p,  L = sum_p 2^(m_p - M) l_p,  out = sum_p 2^(m_p - M) O_p / L.
-// Grid (H, B), one thread per output element of a head.
+// Grid (KV head, sequence), G * D threads: one per output element of the group.
+// It is launched as a programmatic dependent of decode_kernel and waits for it
+// (griddepcontrol.wait) before reading the partials.
 template <typename T>
 __global__ void decode_reduce_kernel(const DecodeParams prm, int D) {
-    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int hk = blockIdx.x, b = blockIdx.y;
+    const int G = prm.num_heads / prm.num_kv_heads;
+    const int g = threadIdx.x / D, d = threadIdx.x % D;
     const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
     const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
     const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
-    if (parts == 1) return;
+    if (parts == 1 || g >= G) return;
+    const int h = hk * G + g;
     const size_t base = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts;
-    float M = -CUDART_INF_F;
-    for (int p = 0; p < parts; ++p) M = fmaxf(M, prm.ws_m[base + p]);
-    float O = 0.f, L = 0.f;
-    for (int p = 0; p < parts; ++p) {
-        const float mp = prm.ws_m[base + p];
-        if (mp == -CUDART_INF_F) continue;
-        const float wt = exp2f(mp - M);
-        L += wt * prm.ws_l[base + p];
-        O += wt * prm.ws_o[(base + p) * D + d];
+    // one pass with a running max: the loads of up to 8 partitions go out together
+    float M = -CUDART_INF_F, O = 0.f, L = 0.f;
+    for (int p0 = 0; p0 < parts; p0 += 8) {
+        float mp[8], lp[8], op[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool in = p0 + i < parts;
+            mp[i] = in ? prm.ws_m[base + p0 + i] : -CUDART_INF_F;
+            lp[i] = in ? prm.ws_l[base + p0 + i] : 0.f;
+            op[i] = in ? prm.ws_o[(base + p0 + i) * D + d] : 0.f;
+        }
+        float mc = M;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
+        if (mc == -CUDART_INF_F) continue;
+        const float a = exp2f(M - mc);  // 0 while M is still -inf
+        O *= a;
+        L *= a;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float wt = mp[i] == -CUDART_INF_F ? 0.f : exp2f(mp[i] - mc);
+            O += wt * op[i];
+            L += wt * lp[i];
+        }
+        M = mc;
     }
     T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
     store_out(out, L > 0.f ? O / L : 0.f);

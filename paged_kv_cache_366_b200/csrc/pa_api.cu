@@ -124,13 +124,27 @@ int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
         !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(T), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
         return PA_ERR_UNSUPPORTED;
-    const dim3 grid(prm.max_parts, prm.num_kv_heads, num_seqs);
-    pa::decode_kernel<T, D, G><<<grid, pa::kDecodeThreads, C::SMEM, st>>>(prm, tm_k, tm_v);
-    int rc = check_launch();
-    if (rc != PA_OK || prm.max_parts == 1) return rc;
-    const dim3 rgrid(prm.num_heads, num_seqs);
-    pa::decode_reduce_kernel<T><<<rgrid, D, 0, st>>>(prm, D);
-    return check_launch();
+    // Both kernels are programmatic dependent launches: each starts launching
+    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
+    // before reading anything.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.num_kv_heads, num_seqs, prm.max_parts);
+    cfg.blockDim = dim3(pa::kDecodeThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<T, D, G>, prm, tm_k, tm_v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (prm.max_parts == 1) return PA_OK;
+    cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
+    cfg.blockDim = dim3(G * D);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<T>, prm, D);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
 template <typename T, int D>
@@ -215,7 +229,7 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     DecodeGeometry g;
     rc = decode_geometry(num_seqs, max_context_len, partition_tokens, shape, &g);
     if (rc != PA_OK) return rc;
-    if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;  // grid z / y limit
+    if (num_seqs > 65535 || g.max_parts > 65535) return PA_ERR_UNSUPPORTED;  // grid y / z limits
     pa::DecodeParams prm{};
     if (g.ws_bytes > 0) {
         if (!workspace || workspace_bytes < g.ws_bytes) return PA_ERR_WORKSPACE;
