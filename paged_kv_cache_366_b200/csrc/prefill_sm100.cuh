@@ -132,25 +132,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 
 // ---- geometry -------------------------------------------------------------------
 
-constexpr int kPfThreads = 256;
-constexpr int kPfM = 128;  // rows per CTA
-constexpr int kPfN = 128;  // keys per tile
-constexpr int kPfD = 128;  // head_dim
-constexpr int kPfHalf = kPfM * 64 * 2;          // one 64-column half of a 128-row bf16 tile: 16 KB
-constexpr int kPfTile = 2 * kPfHalf;            // a 128 x 128 bf16 tile: 32 KB
+constexpr int kPfWarps = 12;
+constexpr int kPfThreads = 32 * kPfWarps;
+constexpr int kPfM = 128;                    // rows per Q tile (tokens x group heads)
+constexpr int kPfNQ = 2;                     // Q tiles per CTA, ping-ponged
+constexpr int kPfN = 64;                     // keys per K/V tile
+constexpr int kPfD = 128;                    // head_dim
+constexpr int kPfNS = 3;                     // K/V pipeline stages
+constexpr int kPfQHalf = kPfM * 64 * 2;      // a 64-column half of a Q tile: 16 KB
+constexpr int kPfQTile = 2 * kPfQHalf;       // 32 KB
+constexpr int kPfKVHalf = kPfN * 64 * 2;     // a 64-dim half of a K/V tile: 8 KB
+constexpr int kPfKVTile = 2 * kPfKVHalf;     // 16 KB
+constexpr int kPfPTile = kPfM * kPfN * 2;    // P: 128 rows x 64 keys bf16 = 16 KB
 constexpr int kPfOffQ = 0;
-constexpr int kPfOffK = kPfOffQ + kPfTile;      // 2 stages
-constexpr int kPfOffV = kPfOffK + 2 * kPfTile;  // 2 stages
-constexpr int kPfOffP = kPfOffV + 2 * kPfTile;
-constexpr int kPfOffBar = kPfOffP + kPfTile;    // mbarriers (8 B each)
-constexpr int kPfBars = 9;                      // q, k[2], v[2], s[2], o, spare
-constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;
-constexpr int kPfOffRed = kPfOffSlot + 16;      // [2][128] floats: row max / row sum halves
-constexpr int kPfSmem = kPfOffRed + 2 * 128 * 4 + 1024;  // + room to align the base to 1024 B
-constexpr uint32_t kPfTmemCols = 512;
-constexpr int kPfBlocksPerTile = kPfN / kBlockSize;
+constexpr int kPfOffK = kPfOffQ + kPfNQ * kPfQTile;
+constexpr int kPfOffV = kPfOffK + kPfNS * kPfKVTile;
+constexpr int kPfOffP = kPfOffV + kPfNS * kPfKVTile;
+constexpr int kPfOffBar = kPfOffP + kPfNQ * kPfPTile;
+// mbarriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], vzero, drain, then per Q tile:
+// sfull, sfree, pready, odone
+constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNS, kPfBarVF = kPfBarKE + kPfNS,
+              kPfBarVE = kPfBarVF + kPfNS, kPfBarVZ = kPfBarVE + kPfNS, kPfBarDrain = kPfBarVZ + 1,
+              kPfBarTile = kPfBarDrain + 1, kPfBars = kPfBarTile + 4 * kPfNQ;
+constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;  // TMEM base address, abort flag
+constexpr int kPfSmem = kPfOffSlot + 16 + 1024;      // + room to align the base to 1024 B
+constexpr uint32_t kPfTmemCols = 512;                // S_A, S_B (64 each), O_A, O_B (128 each)
+constexpr int kPfBlocksPerTile = kPfN / kBlockSize;  // 4
 static_assert(kPfSmem <= 232448, "prefill shared memory over the 227 KB limit");
-static_assert(kPfBlocksPerTile == 8, "warp 0 lanes 0..7 own one block each");
 
 struct PrefillParams {
     void *out;
@@ -165,13 +173,32 @@ struct PrefillParams {
     float scale_log2;
 };
 
+// Bounded mbarrier wait that also gives up when another role of the CTA has aborted.
+__device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            flag_status(PA_STATUS_WAIT_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const PrefillParams prm, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
-    constexpr int TOK = kPfM / G;  // chunk tokens per CTA
+    constexpr int TOK = kPfM / G;  // chunk tokens per Q tile
     const int b = blockIdx.z, hk = blockIdx.y;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+
+    // Launched as a programmatic dependent: wait for the previous kernel (e.g. the
+    // cache write of this chunk) before reading any input.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // ---- per-sequence geometry (uniform over the CTA) ----
     const int q0 = __ldg(prm.cu_q_lens + b), q1 = __ldg(prm.cu_q_lens + b + 1);
@@ -186,282 +213,288 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (first) flag_status(PA_STATUS_BAD_CONTEXT);
         return;
     }
-    const int n_qt = (q_len + TOK - 1) / TOK;
-    const int qt = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // longest tiles launch first
-    if (qt >= n_qt) return;
-    const int t0 = qt * TOK;
+    const int n_ct = (q_len + kPfNQ * TOK - 1) / (kPfNQ * TOK);
+    const int ct = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // longest CTAs first
+    if (ct >= n_ct) return;
+    const int t0 = ct * kPfNQ * TOK;
     const int o = c - q_len;
-    const int rows_valid = min(TOK, q_len - t0);       // chunk tokens of this CTA
-    const int kv_end = o + t0 + rows_valid;            // keys needed: [0, kv_end)
+    const int kv_end = o + min(t0 + kPfNQ * TOK, q_len);  // keys needed: [0, kv_end)
     const int n_tiles = (kv_end + kPfN - 1) / kPfN;
     const int nblk_seq = (c + kBlockSize - 1) / kBlockSize;
+    const bool zero_tail = n_tiles * kPfN > c;  // the last tile holds keys past the context
 
     // ---- shared memory (base aligned to 1024 B for the 128-byte swizzle) ----
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
     unsigned char *base = smem_raw + (base_s - raw_s);
-    const uint32_t sQ = base_s + kPfOffQ, sK = base_s + kPfOffK, sV = base_s + kPfOffV, sP = base_s + kPfOffP;
-    const uint32_t bar_q = base_s + kPfOffBar;
-    const uint32_t bar_k = bar_q + 8;       // [2]
-    const uint32_t bar_v = bar_q + 24;      // [2]
-    const uint32_t bar_s = bar_q + 40;      // [2]
-    const uint32_t bar_o = bar_q + 56;
+    const uint32_t bars = base_s + kPfOffBar;
+    auto bar = [&](int i) -> uint32_t { return bars + 8u * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kPfOffSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + kPfOffSlot + 4);
 
     if (tid == 0) {
-        mbar_init(bar_q, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_k + 8 * i, 1);
-            mbar_init(bar_v + 8 * i, 1);
-            mbar_init(bar_s + 8 * i, 1);
+        mbar_init(bar(kPfBarQ), 1);
+        for (int i = 0; i < kPfNS; ++i) {
+            mbar_init(bar(kPfBarKF + i), 1);
+            mbar_init(bar(kPfBarKE + i), 1);
+            mbar_init(bar(kPfBarVF + i), 1);
+            mbar_init(bar(kPfBarVE + i), 1);
         }
-        mbar_init(bar_o, 1);
+        mbar_init(bar(kPfBarVZ), 1);
+        mbar_init(bar(kPfBarDrain), 1);
+        for (int qi = 0; qi < kPfNQ; ++qi) {
+            mbar_init(bar(kPfBarTile + 4 * qi + 0), 1);    // sfull: MMA commit
+            mbar_init(bar(kPfBarTile + 4 * qi + 1), 128);  // sfree: every softmax thread
+            mbar_init(bar(kPfBarTile + 4 * qi + 2), 128);  // pready: every softmax thread
+            mbar_init(bar(kPfBarTile + 4 * qi + 3), 1);    // odone: MMA commit
+        }
+        *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(smem_addr(tmem_slot), kPfTmemCols);
+    if (warp == 1) tmem_alloc(smem_addr(tmem_slot), kPfTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tO = tmem + 256;  // S tiles at columns 0 and 128
 
-    // ---- loads (warp 0) ----
-    const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq;
-    const int oob_row = static_cast<int>(prm.num_blocks * kBlockSize);  // a row past the pool: TMA fills zeros
-    // pool row of block `lane` (0..7) of tile t, or the out-of-range row
-    auto tile_row = [&](int t) -> int {
-        if (lane >= kPfBlocksPerTile) return oob_row;
-        const int lb = t * kPfBlocksPerTile + lane;
-        if (t >= n_tiles || lb >= nblk_seq) return oob_row;
-        const int pb = __ldg(trow + lb);
-        if (pb < 0 || pb >= prm.num_blocks) {
-            flag_status(PA_STATUS_BAD_BLOCK_ID);
-            return oob_row;
-        }
-        return pb * kBlockSize;
-    };
-    auto load_tile = [&](const CUtensorMap *tm, uint32_t dst, uint32_t bar, int row) {
-        if (lane == 0) mbar_arrive_expect_tx(bar, kPfTile);
-        __syncwarp();
-        if (lane < kPfBlocksPerTile) {
-            const uint32_t d = dst + lane * (kBlockSize * 128);  // 16 rows of 128 B
-            tma_load_3d(d, tm, 0, hk, row, bar);
-            tma_load_3d(d + kPfHalf, tm, 64, hk, row, bar);
-        }
-    };
-    int row_a = 0, row_b = 0, row_c = 0;  // warp 0: pool rows of tiles j+1, j+2, j+3 (row_a = j+1)
     if (warp == 0) {
+        // ================= producer: TMA loads of Q and K/V tiles =================
+        const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq;
+        const int oob_row = static_cast<int>(prm.num_blocks * kBlockSize);  // past the pool: TMA fills zeros
+        auto tile_row = [&](int t) -> int {  // pool row of block `lane` of tile t
+            if (lane >= kPfBlocksPerTile || t >= n_tiles) return oob_row;
+            const int lb = t * kPfBlocksPerTile + lane;
+            if (lb >= nblk_seq) return oob_row;
+            const int pb = __ldg(trow + lb);
+            if (pb < 0 || pb >= prm.num_blocks) {
+                flag_status(PA_STATUS_BAD_BLOCK_ID);
+                return oob_row;
+            }
+            return pb * kBlockSize;
+        };
+        auto load_kv = [&](const CUtensorMap *tm, uint32_t dst, uint32_t full, int row) {
+            if (lane == 0) mbar_arrive_expect_tx(full, kPfKVTile);
+            __syncwarp();
+            if (lane < kPfBlocksPerTile) {
+                const uint32_t d = dst + lane * (kBlockSize * 128);  // 16 rows of 128 B
+                tma_load_3d(d, tm, 0, hk, row, full);
+                tma_load_3d(d + kPfKVHalf, tm, 64, hk, row, full);
+            }
+        };
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar_q, kPfTile);
-            const int qrow = q0 + t0;
-            tma_load_3d(sQ, &tm_q, 0, hk * G, qrow, bar_q);
-            tma_load_3d(sQ + kPfHalf, &tm_q, 64, hk * G, qrow, bar_q);
+            mbar_arrive_expect_tx(bar(kPfBarQ), kPfNQ * kPfQTile);
+            for (int qi = 0; qi < kPfNQ; ++qi) {
+                const uint32_t dq = base_s + kPfOffQ + qi * kPfQTile;
+                const int qrow = q0 + t0 + qi * TOK;
+                tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(kPfBarQ));
+                tma_load_3d(dq + kPfQHalf, &tm_q, 64, hk * G, qrow, bar(kPfBarQ));
+            }
         }
-        const int r0 = tile_row(0);
-        row_a = tile_row(1);
-        row_b = tile_row(2);
-        load_tile(&tm_k, sK, bar_k, r0);
-        load_tile(&tm_v, sV, bar_v, r0);
-        if (n_tiles > 1) {
-            load_tile(&tm_k, sK + kPfTile, bar_k + 8, row_a);
-            load_tile(&tm_v, sV + kPfTile, bar_v + 8, row_a);
-        }
-        row_c = tile_row(3);
-    }
-
-    constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
-    constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
-    // S_t = Q K_t^T into tS[t % 2]
-    auto issue_qk = [&](int t) {
-        const uint32_t kb = sK + (t & 1) * kPfTile;
-#pragma unroll
-        for (int kk = 0; kk < kPfD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPfHalf + (kk & 3) * 32;
-            umma_bf16(tmem + (t & 1) * kPfN, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), kIdQK,
-                      kk > 0);
-        }
-        umma_commit(bar_s + 8 * (t & 1));
-    };
-    // O += P V_t
-    auto issue_pv = [&](int t) {
-        const uint32_t vb = sV + (t & 1) * kPfTile;
-#pragma unroll
-        for (int kk = 0; kk < kPfN / 16; ++kk) {
-            const uint32_t aoff = (kk >> 2) * kPfHalf + (kk & 3) * 32;
-            umma_bf16(tO, smem_desc_sw128(sP + aoff, 16, 1024), smem_desc_sw128(vb + kk * 2048, kPfHalf, 1024), kIdPV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_o);
-    };
-
-    bool ok = true;
-    int qk_issued = 0;  // tid 0 only: QK tiles issued
-    if (tid == 0) {
-        ok = mbar_wait(bar_q, 0) && mbar_wait(bar_k, 0);
-        if (ok) {
-            tc_fence_after();
-            issue_qk(0);
-            qk_issued = 1;
-        }
-    }
-
-    // ---- per-row state: warps w and w+4 share TMEM lanes 32(w%4).., and each takes
-    // one 64-column half of the row (keys of the S tile, dims of O) ----
-    const int quarter = warp & 3, hcol = warp >> 2;
-    const int r = quarter * 32 + lane;
-    const int tok = min(t0 + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
-    const int pos = o + tok;                     // causal limit: keys 0..pos
-    float m_ref = -CUDART_INF_F;                 // reference max (log2 domain) of the row
-    float l_sum = 0.f;                           // this thread's half of the row sum
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    float *red = reinterpret_cast<float *>(base + kPfOffRed);  // [2][128] partial row max, then sums
-    int pv_issued = 0;
-
-    for (int j = 0; j < n_tiles; ++j) {
-        // 1. S_j ready
-        ok = __syncthreads_and(ok ? 1 : 0) != 0;
-        if (!ok) break;
-        bool w = mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1);
-        tc_fence_after();
-        // 2. refill the K stage QK_j just read; issue QK_{j+1}
-        if (warp == 0) {
-            if (j + 2 < n_tiles) load_tile(&tm_k, sK + (j & 1) * kPfTile, bar_k + 8 * (j & 1), row_b);
-            if (tid == 0 && j + 1 < n_tiles && w) {
-                w = mbar_wait(bar_k + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1);
-                if (w) {
-                    tc_fence_after();
-                    issue_qk(j + 1);
-                    qk_issued = j + 2;
+        int row = tile_row(0);
+        int issued = 0;
+        bool ok = true;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+            const int s = j % kPfNS, u = j / kPfNS;
+            const int row_next = tile_row(j + 1);  // fetched while this tile's loads go out
+            if (u >= 1) ok = pf_wait(bar(kPfBarKE + s), (u - 1) & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            load_kv(&tm_k, base_s + kPfOffK + s * kPfKVTile, bar(kPfBarKF + s), row);
+            if (u >= 1) ok = pf_wait(bar(kPfBarVE + s), (u - 1) & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                issued = 2 * j + 1;
+                break;
+            }
+            load_kv(&tm_v, base_s + kPfOffV + s * kPfKVTile, bar(kPfBarVF + s), row);
+            issued = 2 * j + 2;
+            if (j == n_tiles - 1 && zero_tail) {
+                // keys past the context: their V rows (tail slots) may hold anything, and
+                // 0 * NaN would poison O, so zero them before the MMA reads the tile
+                ok = __all_sync(0xffffffffu, pf_wait(bar(kPfBarVF + s), u & 1, abort_flag));
+                if (ok) {
+                    const int first_bad = max(0, c - j * kPfN);
+                    unsigned char *vt = base + kPfOffV + s * kPfKVTile;
+                    for (int i = lane; i < (kPfN - first_bad) * 16; i += 32) {
+                        const int r = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
+                        *reinterpret_cast<uint4 *>(vt + half * kPfKVHalf + r * 128 + chunk * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kPfBarVZ));
                 }
             }
+            row = row_next;
         }
-        // 3. PV_{j-1} done: O stable, P buffer and V stage (j-1)&1 free
-        if (j > 0) {
-            w = mbar_wait(bar_o, (j - 1) & 1) && w;
-            tc_fence_after();
-            if (warp == 0 && j + 1 < n_tiles)
-                load_tile(&tm_v, sV + ((j + 1) & 1) * kPfTile, bar_v + 8 * ((j + 1) & 1), row_a);
-        }
-        if (warp == 0) {  // advance the table window: rows of tiles j+2, j+3, j+4
-            row_a = row_b;
-            row_b = row_c;
-            row_c = tile_row(j + 4);
-        }
-        // 4a. the tile's keys past the context: their V rows (tail slots of the
-        // last block) may hold anything, and 0 * NaN would poison O, so zero them
-        if ((j + 1) * kPfN > c) {
-            w = mbar_wait(bar_v + 8 * (j & 1), (j >> 1) & 1) && w;
-            const int first_bad = max(0, c - j * kPfN);
-            const int n16 = (kPfN - first_bad) * 2 * 8;  // 16-byte chunks in both halves
-            unsigned char *vt = base + kPfOffV + (j & 1) * kPfTile;
-            for (int i = tid; i < n16; i += kPfThreads) {
-                const int row = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
-                *reinterpret_cast<uint4 *>(vt + half * kPfHalf + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        if (*abort_flag) {  // let loads nobody consumed land before the CTA exits
+            for (int i = 0; i < issued; ++i) {
+                const int j = i / 2, s = j % kPfNS, u = j / kPfNS;
+                mbar_wait(bar((i & 1 ? kPfBarVF : kPfBarKF) + s), u & 1);
             }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issue (one thread) =================
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
+            constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
+            auto issue_qk = [&](int qi, int j) {
+                const uint32_t qb = base_s + kPfOffQ + qi * kPfQTile;
+                const uint32_t kb = base_s + kPfOffK + (j % kPfNS) * kPfKVTile;
+#pragma unroll
+                for (int kk = 0; kk < kPfD / 16; ++kk) {
+                    umma_bf16(tmem + qi * kPfN, smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
+                              smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
+                }
+                umma_commit(bar(kPfBarTile + 4 * qi + 0));
+            };
+            auto issue_pv = [&](int qi, int j) {
+                const uint32_t pb = base_s + kPfOffP + qi * kPfPTile;
+                const uint32_t vb = base_s + kPfOffV + (j % kPfNS) * kPfKVTile;
+#pragma unroll
+                for (int kk = 0; kk < kPfN / 16; ++kk) {
+                    umma_bf16(tmem + 2 * kPfN + qi * kPfD, smem_desc_sw128(pb + kk * 32, 16, 1024),
+                              smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar(kPfBarTile + 4 * qi + 3));
+            };
+            bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag) && pf_wait(bar(kPfBarKF), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0, 0);
+                issue_qk(1, 0);
+                umma_commit(bar(kPfBarKE));
+            }
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                const int s = j % kPfNS, u = j / kPfNS;
+                const int s1 = (j + 1) % kPfNS, u1 = (j + 1) / kPfNS;
+                const bool more = j + 1 < n_tiles;
+                for (int qi = 0; qi < kPfNQ && ok; ++qi) {
+                    // S of the next tile once softmax qi has read this tile's S
+                    if (more) {
+                        ok = pf_wait(bar(kPfBarKF + s1), u1 & 1, abort_flag) &&
+                             pf_wait(bar(kPfBarTile + 4 * qi + 1), j & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(qi, j + 1);
+                        if (qi == kPfNQ - 1) umma_commit(bar(kPfBarKE + s1));
+                    }
+                    // O += P V once softmax qi has written P (and rescaled O)
+                    ok = pf_wait(bar(kPfBarTile + 4 * qi + 2), j & 1, abort_flag);
+                    if (ok && qi == 0)
+                        ok = (j == n_tiles - 1 && zero_tail) ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
+                                                             : pf_wait(bar(kPfBarVF + s), u & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(qi, j);
+                    if (qi == kPfNQ - 1) umma_commit(bar(kPfBarVE + s));
+                }
+            }
+            // every MMA issued so far completes before tensor memory can be freed
+            umma_commit(bar(kPfBarDrain));
+            mbar_wait(bar(kPfBarDrain), 0);
         }
         __syncwarp();
-        // 4b. this thread's 64 scores of row r
-        constexpr int HN = kPfN / 2;
-        float s[HN];
-        const uint32_t s_cols = tmem + (j & 1) * kPfN + hcol * HN;
-#pragma unroll
-        for (int ch = 0; ch < HN / 32; ++ch) {
-            float v[32];
-            tmem_ld32(s_cols + lane_base + ch * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[ch * 32 + i] = v[i] * prm.scale_log2;
-        }
-        const int key0 = j * kPfN + hcol * HN;
-        if (key0 + HN - 1 > pos) {
-#pragma unroll
-            for (int i = 0; i < HN; ++i)
-                if (key0 + i > pos) s[i] = -CUDART_INF_F;
-        }
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-        for (int i = 8; i < HN; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
-        const float mx_half = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        red[hcol * kPfM + r] = mx_half;
-        __syncthreads();
-        const float mx = fmaxf(red[r], red[kPfM + r]);
-        float alpha = 1.f;
-        if (mx > m_ref + 8.f || m_ref == -CUDART_INF_F) {
-            const float m_new = fmaxf(mx, m_ref);
-            alpha = (m_ref == -CUDART_INF_F) ? 0.f : exp2f(m_ref - m_new);
-            m_ref = m_new;
-        }
-        float a8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a8[i] = 0.f;
-        unsigned char *prow = base + kPfOffP + hcol * kPfHalf + r * 128;
-#pragma unroll
-        for (int cc = 0; cc < HN / 8; ++cc) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float p0 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[cc * 8 + 2 * e] - m_ref);
-                const float p1 = m_ref == -CUDART_INF_F ? 0.f : exp2f(s[cc * 8 + 2 * e + 1] - m_ref);
-                const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                a8[(2 * e) & 7] += __low2float(pb);
-                a8[(2 * e + 1) & 7] += __high2float(pb);
-                pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
-            }
-            *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-        const float psum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-        l_sum = l_sum * alpha + psum;
-        // rescale this thread's half of O's row in tensor memory (warp-uniform:
-        // tcgen05.ld/st are .sync.aligned)
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-            for (int ch = 0; ch < HN / 32; ++ch) {
-                const uint32_t oc = tO + hcol * HN + lane_base + ch * 32;
-                float v[32];
-                tmem_ld32(oc, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                tmem_st32(oc, v);
-            }
-        }
-        // 5. P visible to the tensor core, TMEM reads/writes ordered before the next MMA
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(w ? 1 : 0) != 0;
-        if (!ok) break;
-        // 6. O += P V_j
-        if (tid == 0) {
+    } else if (warp >= 4) {
+        // ================= softmax: warps 4..7 own Q tile 0, warps 8..11 Q tile 1 =================
+        const int qi = (warp - 4) / 4;
+        const int r = (warp & 3) * 32 + lane;  // row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + qi * kPfN, tO = tmem + 2 * kPfN + qi * kPfD;
+        const uint32_t b_sfull = bar(kPfBarTile + 4 * qi + 0), b_sfree = bar(kPfBarTile + 4 * qi + 1);
+        const uint32_t b_pready = bar(kPfBarTile + 4 * qi + 2), b_odone = bar(kPfBarTile + 4 * qi + 3);
+        const int tq = t0 + qi * TOK;                 // first chunk token of this Q tile
+        const int rows_valid = max(0, min(TOK, q_len - tq));
+        const int tok = min(tq + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
+        const int pos = o + tok;                      // causal limit: keys 0..pos
+        unsigned char *prow = base + kPfOffP + qi * kPfPTile + r * 128;
+        float m_ref = -CUDART_INF_F, l_sum = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            ok = __all_sync(0xffffffffu, pf_wait(b_sfull, j & 1, abort_flag));
+            if (!ok) break;
             tc_fence_after();
-            if (mbar_wait(bar_v + 8 * (j & 1), (j >> 1) & 1)) {
-                issue_pv(j);
-            } else {
-                ok = false;
-            }
-        }
-        pv_issued = j + 1;
-    }
-    ok = __syncthreads_and(ok ? 1 : 0) != 0;
-
-    // ---- epilogue: out = O / l for the valid rows, each thread its 64 dims ----
-    if (ok && pv_issued == n_tiles && n_tiles > 0) {
-        red[hcol * kPfM + r] = l_sum;
-        ok = mbar_wait(bar_o, (n_tiles - 1) & 1);
-        ok = __syncthreads_and(ok ? 1 : 0) != 0;
-        tc_fence_after();
-        if (ok) {
-            const float l_row = red[r] + red[kPfM + r];
-            const bool row_ok = r / G < rows_valid;
-            const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
-            const int orow = row_ok ? q0 + t0 + r / G : q0;
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
-                                 (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD + hcol * 64;
+            float s[kPfN];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < kPfN / 32; ++ch) {
                 float v[32];
-                tmem_ld32(tO + hcol * 64 + lane_base + ch * 32, v);
+                tmem_ld32(tS + lane_base + ch * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s[ch * 32 + i] = v[i] * prm.scale_log2;
+            }
+            tc_fence_before();
+            mbar_arrive(b_sfree);  // S may be overwritten by the next QK
+            const int key0 = j * kPfN;
+            if (key0 + kPfN - 1 > pos) {
+#pragma unroll
+                for (int i = 0; i < kPfN; ++i)
+                    if (key0 + i > pos) s[i] = -CUDART_INF_F;
+            }
+            float m8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+            for (int i = 8; i < kPfN; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            float alpha = 1.f;
+            if (mx > m_ref + 8.f) {  // lazy: keep the older max unless a score exceeds it by 2^8
+                alpha = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
+                m_ref = mx;
+            }
+            // PV of the previous tile done: O is stable and the P buffer is free
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, pf_wait(b_odone, (j - 1) & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
+#pragma unroll
+                    for (int ch = 0; ch < kPfD / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(tO + lane_base + ch * 32, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                        tmem_st32(tO + lane_base + ch * 32, v);
+                    }
+                }
+            }
+            float a8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a8[i] = 0.f;
+            const bool live = m_ref != -CUDART_INF_F;
+#pragma unroll
+            for (int cc = 0; cc < kPfN / 8; ++cc) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = live ? exp2f(s[cc * 8 + 2 * e] - m_ref) : 0.f;
+                    const float p1 = live ? exp2f(s[cc * 8 + 2 * e + 1] - m_ref) : 0.f;
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    a8[2 * e] += __low2float(pb);
+                    a8[2 * e + 1] += __high2float(pb);
+                    pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+                *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            l_sum = l_sum * alpha + (((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7])));
+            fence_async_smem();  // P visible to the tensor core
+            tc_fence_before();
+            mbar_arrive(b_pready);
+        }
+        // ---- epilogue: out = O / l for the valid rows ----
+        if (ok) ok = __all_sync(0xffffffffu, pf_wait(b_odone, (n_tiles - 1) & 1, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            const bool row_ok = r / G < rows_valid;
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const int orow = row_ok ? q0 + tq + r / G : q0;
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
+                                 (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
+#pragma unroll
+            for (int ch = 0; ch < kPfD / 32; ++ch) {
+                float v[32];
+                tmem_ld32(tO + lane_base + ch * 32, v);
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) {
                     uint4 pkt;
@@ -477,14 +510,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
             }
         }
-    } else if (tid == 0) {
-        // failed: let the MMAs already issued finish before tensor memory is freed
-        if (pv_issued > 0) mbar_wait(bar_o, (pv_issued - 1) & 1);
-        if (qk_issued > 0) mbar_wait(bar_s + 8 * ((qk_issued - 1) & 1), ((qk_issued - 1) >> 1) & 1);
+        tc_fence_before();
     }
-    tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kPfTmemCols);
     }
@@ -509,10 +538,18 @@ int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cach
             return PA_ERR_CUDA;
         attr_done[dev] = true;
     }
-    const int n_qt = (max_q_len + TOK - 1) / TOK;
-    const dim3 grid(n_qt, s->num_kv_heads, num_seqs);
-    prefill_kernel<G><<<grid, kPfThreads, kPfSmem, st>>>(prm, tm_q, tm_k, tm_v);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const int n_ct = (max_q_len + kPfNQ * TOK - 1) / (kPfNQ * TOK);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_ct, s->num_kv_heads, num_seqs);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = kPfSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<G>, prm, tm_q, tm_k, tm_v) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 inline int launch_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
