@@ -172,8 +172,10 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
  *   cu_q_lens    : int32 [B + 1] device, non-decreasing, cu_q_lens[0] = 0
  *   context_lens : int32 [B] device, >= q_len
  *   max_q_len    : host-side upper bound of every q_len (sizes the grid)
+ *   scale        : softmax scale, > 0 (PA_ERR_INVALID_ARGUMENT otherwise)
  * bf16 only, D = 128 only. Runs on the tcgen05 tensor cores with fp32
- * accumulation in tensor memory. Returns PA_ERR_UNSUPPORTED otherwise.
+ * accumulation in tensor memory. Probabilities enter P.V rounded to bf16;
+ * the row sums use them unrounded. Returns PA_ERR_UNSUPPORTED otherwise.
  */
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *cu_q_lens,

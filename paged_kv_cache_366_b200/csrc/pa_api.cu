@@ -275,7 +275,7 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
     if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens)
         return PA_ERR_INVALID_ARGUMENT;
-    if (max_blocks_per_seq < 1 || !std::isfinite(scale)) return PA_ERR_INVALID_ARGUMENT;
+    if (max_blocks_per_seq < 1 || !std::isfinite(scale) || !(scale > 0.f)) return PA_ERR_INVALID_ARGUMENT;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_tables, 4) ||
         !aligned(cu_q_lens, 4) || !aligned(context_lens, 4))
         return PA_ERR_ALIGNMENT;

@@ -130,6 +130,17 @@ __device__ __forceinline__ void fma2(f32x2 &d, f32x2 a, f32x2 b) {
 // d *= a
 __device__ __forceinline__ void mul2(f32x2 &d, f32x2 a) { asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a)); }
 
+// d += a
+__device__ __forceinline__ void add2(f32x2 &d, f32x2 a) { asm("add.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a)); }
+
+// 2^x with the hardware approximation (ex2.approx.ftz.f32): 2^-inf = 0,
+// subnormal results flush to zero. Used where the result is rounded to bf16.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Widen 16 bytes of storage to fp32: 8 bf16 or 4 fp32 values.
 template <typename T>
 struct Widen;

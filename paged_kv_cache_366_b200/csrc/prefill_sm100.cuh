@@ -8,31 +8,35 @@
 //   out[j][h] = softmax_k(scale * q[j][h] . K[k]) V[k],  k <= o + j,
 // with K/V rows found through the block table, as in decode.
 //
-// How it runs (bf16 in, fp32 accumulate, head_dim 128):
-//  * A CTA owns 128 rows = (128 / G) chunk tokens x the G query heads of one KV
-//    head (GQA packing), so every K/V tile loaded serves all G heads.
-//  * Q (128 x 128) and each K/V tile (128 keys x 128) come in by TMA with
-//    128-byte swizzle. A K/V tile is eight 16-token blocks; each block of each
-//    64-column half is one TMA box addressed through the block table. Blocks
-//    past the context (and bad table entries) load from an out-of-range
-//    coordinate, which fills zeros.
-//  * S = Q K^T and O += P V run on the tensor cores (tcgen05.mma kind::f16,
-//    M=128, N=128, K=16 per instruction) with accumulators in tensor memory:
-//    two S buffers and one O, 384 of the 512 columns. QK of tile j+1 is issued
-//    before the softmax of tile j, so the two overlap.
-//  * Softmax: 8 warps. The two warps that share a TMEM lane quarter split each
-//    row into 64-column halves and exchange partial maxima and sums through
-//    shared memory. They mask keys past the row's causal limit and keep a
-//    running max in the exp2 domain, with tree-shaped max/sum reductions. P goes
-//    as bf16 into shared memory in the 128-byte-swizzled K-major layout the MMA
-//    reads. O is rescaled in TMEM only when the row max grows by more than
-//    2^8; otherwise the older max is kept, and P stays below 256.
-//  * One thread issues the MMAs and commits them to mbarriers. Warp 0's lanes
-//    0..7 issue the TMA loads, one block each. The table entries for a tile are
-//    fetched one iteration before its loads.
-//  * Every mbarrier wait is bounded. On a timeout the CTA flags
-//    PA_STATUS_WAIT_TIMEOUT, waits (bounded) for its in-flight MMAs, frees its
-//    tensor memory and returns.
+// How it runs (bf16 in, fp32 accumulate, head_dim 128), warp-specialized:
+//  * A CTA owns two Q tiles of 128 rows. Each row is one of (128 / G) chunk
+//    tokens x the G query heads of one KV head (GQA packing), so every K/V tile
+//    loaded serves all G heads of both Q tiles.
+//  * Warp 0 (producer) streams Q and then 64-key K/V tiles by TMA with 128-byte
+//    swizzle into a 3-stage ring. A tile is four 16-token blocks, and each block
+//    of each 64-column half is one TMA box addressed through the block table.
+//    Blocks past the context (and bad table entries) load from an out-of-range
+//    row, which fills zeros. The producer zeroes the last tile's V rows past the
+//    context before the MMA may read them (0 * NaN would poison O).
+//  * Warp 1 issues the MMAs from one thread: S = Q K^T (M=128, N=64) and
+//    O += P V (M=128, N=128), tcgen05.mma kind::f16, with S and O for both Q
+//    tiles in tensor memory. The order is QK(tile 0, j+1), PV(tile 0, j),
+//    QK(tile 1, j+1), PV(tile 1, j), so one Q tile's softmax overlaps the other
+//    tile's MMAs.
+//  * Warps 4..7 and 8..11 run the softmax of Q tiles 0 and 1; thread = row =
+//    TMEM lane. A thread reads its 64 scores in one tcgen05.ld and releases S
+//    at once. It masks keys past its causal limit, takes the row max, and
+//    computes p = 2^(s*scale*log2(e) - m) with one FMA and one ex2. It writes
+//    P as bf16 into shared memory in the swizzled K-major layout the MMA reads,
+//    and sums the fp32 p in packed pairs. The reference max is replaced (and O
+//    rescaled in TMEM) only when a row max grows by more than 2^8.
+//  * P is double-buffered per Q tile. The softmax of tile j waits only for the
+//    PV of tile j-2 (buffer reuse), and for that of tile j-1 only when it
+//    rescales O.
+//  * Hand-offs are mbarriers only: full/empty per ring stage (empties committed
+//    by tcgen05.commit), sfull/sfree for S, pready, and odone per P buffer.
+//    Every wait is bounded and also gives up when another role has aborted. The
+//    MMA thread drains its work before tensor memory is freed.
 #pragma once
 
 #include <math_constants.h>
@@ -89,6 +93,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane, one load instruction.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, "
+        "%36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, "
+        "%57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -148,12 +174,12 @@ constexpr int kPfOffQ = 0;
 constexpr int kPfOffK = kPfOffQ + kPfNQ * kPfQTile;
 constexpr int kPfOffV = kPfOffK + kPfNS * kPfKVTile;
 constexpr int kPfOffP = kPfOffV + kPfNS * kPfKVTile;
-constexpr int kPfOffBar = kPfOffP + kPfNQ * kPfPTile;
+constexpr int kPfOffBar = kPfOffP + 2 * kPfNQ * kPfPTile;  // P double-buffered per Q tile
 // mbarriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], vzero, drain, then per Q tile:
-// sfull, sfree, pready, odone
+// sfull, sfree, pready, odone[2] (one per P buffer)
 constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNS, kPfBarVF = kPfBarKE + kPfNS,
               kPfBarVE = kPfBarVF + kPfNS, kPfBarVZ = kPfBarVE + kPfNS, kPfBarDrain = kPfBarVZ + 1,
-              kPfBarTile = kPfBarDrain + 1, kPfBars = kPfBarTile + 4 * kPfNQ;
+              kPfBarTile = kPfBarDrain + 1, kPfTileBars = 5, kPfBars = kPfBarTile + kPfTileBars * kPfNQ;
 constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;  // TMEM base address, abort flag
 constexpr int kPfSmem = kPfOffSlot + 16 + 1024;      // + room to align the base to 1024 B
 constexpr uint32_t kPfTmemCols = 512;                // S_A, S_B (64 each), O_A, O_B (128 each)
@@ -244,10 +270,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_init(bar(kPfBarVZ), 1);
         mbar_init(bar(kPfBarDrain), 1);
         for (int qi = 0; qi < kPfNQ; ++qi) {
-            mbar_init(bar(kPfBarTile + 4 * qi + 0), 1);    // sfull: MMA commit
-            mbar_init(bar(kPfBarTile + 4 * qi + 1), 128);  // sfree: every softmax thread
-            mbar_init(bar(kPfBarTile + 4 * qi + 2), 128);  // pready: every softmax thread
-            mbar_init(bar(kPfBarTile + 4 * qi + 3), 1);    // odone: MMA commit
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 0), 1);    // sfull: MMA commit
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // sfree: every softmax thread
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 2), 128);  // pready: every softmax thread
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 3), 1);    // odone, P buffer 0: MMA commit
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 4), 1);    // odone, P buffer 1: MMA commit
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -347,17 +374,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     umma_bf16(tmem + qi * kPfN, smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
                               smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
                 }
-                umma_commit(bar(kPfBarTile + 4 * qi + 0));
+                umma_commit(bar(kPfBarTile + kPfTileBars * qi + 0));
             };
             auto issue_pv = [&](int qi, int j) {
-                const uint32_t pb = base_s + kPfOffP + qi * kPfPTile;
+                const uint32_t pb = base_s + kPfOffP + (2 * qi + (j & 1)) * kPfPTile;
                 const uint32_t vb = base_s + kPfOffV + (j % kPfNS) * kPfKVTile;
 #pragma unroll
                 for (int kk = 0; kk < kPfN / 16; ++kk) {
                     umma_bf16(tmem + 2 * kPfN + qi * kPfD, smem_desc_sw128(pb + kk * 32, 16, 1024),
                               smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(bar(kPfBarTile + 4 * qi + 3));
+                umma_commit(bar(kPfBarTile + kPfTileBars * qi + 3 + (j & 1)));
             };
             bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag) && pf_wait(bar(kPfBarKF), 0, abort_flag);
             if (ok) {
@@ -374,14 +401,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     // S of the next tile once softmax qi has read this tile's S
                     if (more) {
                         ok = pf_wait(bar(kPfBarKF + s1), u1 & 1, abort_flag) &&
-                             pf_wait(bar(kPfBarTile + 4 * qi + 1), j & 1, abort_flag);
+                             pf_wait(bar(kPfBarTile + kPfTileBars * qi + 1), j & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         issue_qk(qi, j + 1);
                         if (qi == kPfNQ - 1) umma_commit(bar(kPfBarKE + s1));
                     }
                     // O += P V once softmax qi has written P (and rescaled O)
-                    ok = pf_wait(bar(kPfBarTile + 4 * qi + 2), j & 1, abort_flag);
+                    ok = pf_wait(bar(kPfBarTile + kPfTileBars * qi + 2), j & 1, abort_flag);
                     if (ok && qi == 0)
                         ok = (j == n_tiles - 1 && zero_tail) ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
                                                              : pf_wait(bar(kPfBarVF + s), u & 1, abort_flag);
@@ -402,27 +429,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int r = (warp & 3) * 32 + lane;  // row = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + qi * kPfN, tO = tmem + 2 * kPfN + qi * kPfD;
-        const uint32_t b_sfull = bar(kPfBarTile + 4 * qi + 0), b_sfree = bar(kPfBarTile + 4 * qi + 1);
-        const uint32_t b_pready = bar(kPfBarTile + 4 * qi + 2), b_odone = bar(kPfBarTile + 4 * qi + 3);
+        const uint32_t b_sfull = bar(kPfBarTile + kPfTileBars * qi + 0);
+        const uint32_t b_sfree = bar(kPfBarTile + kPfTileBars * qi + 1);
+        const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 2);
+        // odone[x] completes when the PV that read P buffer x is done (every other tile)
+        auto b_odone = [&](int x) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + 3 + x); };
         const int tq = t0 + qi * TOK;                 // first chunk token of this Q tile
         const int rows_valid = max(0, min(TOK, q_len - tq));
         const int tok = min(tq + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
         const int pos = o + tok;                      // causal limit: keys 0..pos
-        unsigned char *prow = base + kPfOffP + qi * kPfPTile + r * 128;
+        unsigned char *prow0 = base + kPfOffP + 2 * qi * kPfPTile + r * 128;
         float m_ref = -CUDART_INF_F, l_sum = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             ok = __all_sync(0xffffffffu, pf_wait(b_sfull, j & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float s[kPfN];
-#pragma unroll
-            for (int ch = 0; ch < kPfN / 32; ++ch) {
-                float v[32];
-                tmem_ld32(tS + lane_base + ch * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) s[ch * 32 + i] = v[i] * prm.scale_log2;
-            }
+            float s[kPfN];  // raw q.k; scale (> 0) is applied inside the exponent
+            tmem_ld64(tS + lane_base, s);
             tc_fence_before();
             mbar_arrive(b_sfree);  // S may be overwritten by the next QK
             const int key0 = j * kPfN;
@@ -437,18 +461,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int i = 8; i < kPfN; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * prm.scale_log2;
             float alpha = 1.f;
             if (mx > m_ref + 8.f) {  // lazy: keep the older max unless a score exceeds it by 2^8
                 alpha = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
                 m_ref = mx;
             }
-            // PV of the previous tile done: O is stable and the P buffer is free
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, pf_wait(b_odone, (j - 1) & 1, abort_flag));
+            // a rescale needs O stable: the PV of tile j-1 (P buffer (j-1)&1) done
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
+                ok = __all_sync(0xffffffffu, pf_wait(b_odone((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
+                {
 #pragma unroll
                     for (int ch = 0; ch < kPfD / 32; ++ch) {
                         float v[32];
@@ -459,31 +483,42 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
             }
-            float a8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) a8[i] = 0.f;
-            const bool live = m_ref != -CUDART_INF_F;
+            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score; the row sum
+            // accumulates the fp32 p in packed pairs
+            // P buffer j&1 is free once the PV of tile j-2 is done
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu, pf_wait(b_odone(j & 1), ((j >> 1) - 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+            unsigned char *prow = prow0 + (j & 1) * kPfPTile;
+            const float nm = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+            const float sc = m_ref == -CUDART_INF_F ? 0.f : prm.scale_log2;
+            f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int cc = 0; cc < kPfN / 8; ++cc) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = live ? exp2f(s[cc * 8 + 2 * e] - m_ref) : 0.f;
-                    const float p1 = live ? exp2f(s[cc * 8 + 2 * e + 1] - m_ref) : 0.f;
+                    const float p0 = ex2_approx(fmaf(s[cc * 8 + 2 * e], sc, nm));
+                    const float p1 = ex2_approx(fmaf(s[cc * 8 + 2 * e + 1], sc, nm));
+                    add2(acc[e], pack2(p0, p1));
                     const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    a8[2 * e] += __low2float(pb);
-                    a8[2 * e + 1] += __high2float(pb);
                     pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
                 }
                 *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            l_sum = l_sum * alpha + (((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7])));
+            add2(acc[0], acc[1]);
+            add2(acc[2], acc[3]);
+            add2(acc[0], acc[2]);
+            float lo, hi;
+            unpack2(acc[0], lo, hi);
+            l_sum = l_sum * alpha + (lo + hi);
             fence_async_smem();  // P visible to the tensor core
             tc_fence_before();
             mbar_arrive(b_pready);
         }
         // ---- epilogue: out = O / l for the valid rows ----
-        if (ok) ok = __all_sync(0xffffffffu, pf_wait(b_odone, (n_tiles - 1) & 1, abort_flag));
+        if (ok) ok = __all_sync(0xffffffffu, pf_wait(b_odone((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, abort_flag));
         if (ok) {
             tc_fence_after();
             const bool row_ok = r / G < rows_valid;
