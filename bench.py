@@ -47,7 +47,10 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
-WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny"]
+WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny",
+             "copy_blocks", "swap_blocks"]
+BLOCK_WORKLOADS = ("copy_blocks", "swap_blocks")
+BLOCK_PAIRS = 2048
 
 
 # ---------------------------------------------------------------------------
@@ -563,6 +566,109 @@ def run_ours(args):
     return 0
 
 
+def run_blocks(args):
+    """Whole-block copies on the decode-batch pool.
+
+    copy_blocks: copy-on-write of 2048 (used -> free) blocks, K and V, inside HBM.
+    swap_blocks: 2048 blocks of K and V out to pinned host memory and back in,
+    one pa_swap_blocks launch per pool and direction.
+    """
+    import torch
+    from paged_kv_cache_366_b200 import pa
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
+        return 0  # replicas of a copy measure nothing the single run does not
+    case = W.decode_batch()
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+    k_cache, v_cache = dev(case.k_cache), dev(case.v_cache)
+    rng = np.random.default_rng(17)
+    used = np.unique(case.block_tables[case.block_tables >= 0])
+    free = np.setdiff1d(np.arange(case.num_blocks), used)
+    n = min(BLOCK_PAIRS, len(free))
+    block_bytes = k_cache[0].numel() * 2
+    stream = torch.cuda.Stream()
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    if args.workload == "copy_blocks":
+        pairs = torch.from_numpy(np.stack([rng.choice(used, n), rng.choice(free, n, replace=False)], 1)
+                                 .astype(np.int64)).cuda()
+        fns = [lambda: pa.pa_copy_blocks(k_cache, v_cache, pairs)]
+        nbytes = n * 2 * 2 * block_bytes
+        launches = 2
+        peak, kind = load_peak()
+        bound, peak_note = "hbm", kind + " (MEASURED_PEAKS.json hbm_gbs)"
+    else:
+        src_ids = rng.choice(used, n, replace=False)
+        host_k = torch.empty((n,) + tuple(k_cache.shape[1:]), dtype=torch.bfloat16).pin_memory()
+        host_v = torch.empty_like(host_k).pin_memory()
+        out_pairs = torch.from_numpy(np.stack([src_ids, np.arange(n)], 1).astype(np.int64)).cuda()
+        in_pairs = torch.from_numpy(np.stack([np.arange(n), rng.choice(free, n, replace=False)], 1)
+                                    .astype(np.int64)).cuda()
+        fns = [lambda: (pa.pa_swap_blocks(host_k, k_cache, out_pairs), pa.pa_swap_blocks(host_v, v_cache, out_pairs),
+                        pa.pa_swap_blocks(k_cache, host_k, in_pairs), pa.pa_swap_blocks(v_cache, host_v, in_pairs))]
+        nbytes = n * 2 * 2 * block_bytes  # out and back in, K and V, over the host link
+        launches = 4
+        # link reference, measured here: contiguous pinned copies of the same bytes, out and in
+        dbuf = torch.empty(n * block_bytes, dtype=torch.uint8, device="cuda")
+        hbuf = torch.empty(n * block_bytes, dtype=torch.uint8).pin_memory()
+        ts = []
+        with torch.cuda.stream(stream):
+            for i in range(6):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(2):
+                    hbuf.copy_(dbuf, non_blocking=True)
+                    dbuf.copy_(hbuf, non_blocking=True)
+                e1.record(stream)
+                stream.synchronize()
+                if i >= 2:
+                    ts.append(e0.elapsed_time(e1) * 1e-3)
+        peak = 4 * n * block_bytes / statistics.median(ts) / 1e9
+        bound, peak_note = "link", "measured in this run: contiguous pinned cudaMemcpyAsync, same bytes, out and in"
+    with torch.cuda.stream(stream):
+        for f in fns:
+            f()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for f in fns:
+                f()
+        for _ in range(args.warmup):
+            flush_w.zero_()
+            torch.sum(flush_r)
+            g.replay()
+    torch.cuda.synchronize()
+    if pa.pa_get_status(stream):
+        raise SystemExit("device status set by the block copies")
+    sampler = ClockSampler(gpu_id_for(int(os.environ.get("LOCAL_RANK", "0"))))
+    sampler.wait_ready()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for a, b in ev:
+            flush_w.zero_()
+            torch.sum(flush_r)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    t = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
+    value = nbytes / t / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; see paged_kv_cache_366_b200/workloads.py)",
+            "config": {"workload": args.workload, "pool": "decode_batch (seed 1)", "block_pairs": n,
+                       "block_bytes_per_pool": block_bytes,
+                       "l2": "flushed before every step, outside the events (memset then read)"},
+            "roofline": {"bound": bound, "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
+                         "traffic": None, "kernel": "copy_blocks_kernel", "peak_kind": peak_note},
+            "cpu_baseline": None, "e2e": None, "clocks": sampler.summary(wall0, wall1),
+            "gpu_launches": launches * args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -576,7 +682,11 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
+        if args.workload in BLOCK_WORKLOADS:
+            raise SystemExit("the reference arm times the attention step; block copies have no oracle timing")
         return run_reference(args)
+    if args.workload in BLOCK_WORKLOADS:
+        return run_blocks(args)
     return run_ours(args)
 
 

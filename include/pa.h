@@ -183,6 +183,42 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
                      float scale, const pa_shape *shape, void *stream);
 
 /*
+ * pa_copy_blocks: copy whole blocks inside the pool (copy-on-write of shared
+ * prefix blocks: "vLLM — PagedAttention and Continuous Batching" §2.3,
+ * "vLLM and PagedAttention" §2 "The PagedAttention Solution", "How vLLM
+ * Works?" §03).
+ *
+ * For each pair i: block block_pairs[2i+1] of k_cache and of v_cache becomes
+ * a byte copy of block block_pairs[2i]. A block is [16][Hk][D] elements.
+ *   block_pairs : int64 [num_pairs][2] (src, dst), device memory
+ * Destinations must be distinct and no block may be both a source and a
+ * destination in one call (pairs run concurrently). An index outside
+ * [0, NB) skips that pair and sets PA_STATUS_BAD_BLOCK_ID.
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pairs, int64_t num_pairs,
+                   const pa_shape *shape, void *stream);
+
+/*
+ * pa_swap_blocks: move whole blocks of one pool between device memory and
+ * pinned host memory, either way (preemption by swapping: "vLLM and
+ * PagedAttention" §3, "How vLLM Works?" §04).
+ *
+ * For each pair i: block block_pairs[2i+1] of dst becomes a byte copy of block
+ * block_pairs[2i] of src. Call once for K and once for V.
+ *   dst, src    : device memory or pinned (page-locked) host memory; the kernel
+ *                 reaches host memory through its device mapping, so the whole
+ *                 swap is one launch. Pageable host memory is refused
+ *                 (PA_ERR_INVALID_ARGUMENT).
+ *   block_pairs : int64 [num_pairs][2] (src, dst), device or pinned host memory
+ *   src_blocks, dst_blocks : blocks in each pool; block_bytes : bytes per block
+ *                 (a multiple of 16)
+ * Destinations must be distinct. An index outside its pool skips that pair
+ * and sets PA_STATUS_BAD_BLOCK_ID.
+ */
+int pa_swap_blocks(void *dst, const void *src, const int64_t *block_pairs, int64_t num_pairs, int64_t src_blocks,
+                   int64_t dst_blocks, int64_t block_bytes, void *stream);
+
+/*
  * pa_decode_noalloc: pa_decode for callers that cannot allocate device memory.
  * The paper has no counterpart to this call; it is a deployment convenience.
  *

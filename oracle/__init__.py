@@ -54,6 +54,10 @@ def _load():
             lib.pa_oracle_slot_of.restype = L
             lib.pa_oracle_blocks_for.argtypes = [L, I]
             lib.pa_oracle_blocks_for.restype = L
+            lib.pa_oracle_copy_blocks.argtypes = [P, P, P, L, L, L]
+            lib.pa_oracle_copy_blocks.restype = I
+            lib.pa_oracle_swap_blocks.argtypes = [P, P, P, L, L, L, L]
+            lib.pa_oracle_swap_blocks.restype = I
             lib.pa_oracle_set_mutation.argtypes = [I]
             lib.pa_oracle_set_mutation.restype = None
             lib.pa_oracle_get_mutation.argtypes = []
@@ -179,3 +183,28 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping):
     if n < 0:
         raise OracleError("slot outside the pool")
     return kc, vc
+
+
+def copy_blocks(k_cache, v_cache, pairs):
+    """Return copies of (k_cache, v_cache) where block dst of each (src, dst) pair, in order, copies block src."""
+    kc = np.array(k_cache, copy=True, order="C")
+    vc = np.array(v_cache, copy=True, order="C")
+    pr = _c(pairs, np.int64).reshape(-1, 2)
+    NB = kc.shape[0]
+    bb = kc[0].nbytes
+    rc = _load().pa_oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(pr), pr.shape[0], NB, bb)
+    if rc:
+        raise OracleError("block index outside the pool")
+    return kc, vc
+
+
+def swap_blocks(dst, src, pairs):
+    """Return a copy of dst where block dst_id of each (src_id, dst_id) pair copies block src_id of src."""
+    d = np.array(dst, copy=True, order="C")
+    sr = _c(src)
+    pr = _c(pairs, np.int64).reshape(-1, 2)
+    assert d.dtype == sr.dtype and d.shape[1:] == sr.shape[1:]
+    rc = _load().pa_oracle_swap_blocks(_ptr(d), _ptr(sr), _ptr(pr), pr.shape[0], sr.shape[0], d.shape[0], d[0].nbytes)
+    if rc:
+        raise OracleError("block index outside a pool")
+    return d

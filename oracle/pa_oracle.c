@@ -342,3 +342,47 @@ long pa_oracle_reshape_and_cache(const void *k, const void *v, void *k_cache, vo
     }
     return written;
 }
+
+/*
+ * Block copies. The pages share identical prefixes by pointing several tables
+ * at the same physical blocks and copy a block before it is written
+ * (copy-on-write: "vLLM — PagedAttention and Continuous Batching" §2.3,
+ * "vLLM and PagedAttention" §2 "The PagedAttention Solution", "How vLLM
+ * Works?" §03). Preemption moves a request's blocks out to host memory and
+ * back ("vLLM and PagedAttention" §3; "How vLLM Works?" §04).
+ *
+ * pa_oracle_copy_blocks: for each pair i in order, block pairs[2i+1] of both
+ * pools becomes a byte copy of block pairs[2i]. block_bytes is one block of
+ * one pool (block_size * kv_heads * head_dim * elem). Returns 0, or -1 (and
+ * copies nothing) if an index is outside [0, num_blocks).
+ */
+int pa_oracle_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, long num_pairs, long num_blocks,
+                          long block_bytes)
+{
+    for (long i = 0; i < 2 * num_pairs; ++i)
+        if (pairs[i] < 0 || pairs[i] >= num_blocks)
+            return -1;
+    for (long i = 0; i < num_pairs; ++i) {
+        long src = pairs[2 * i], dst = pairs[2 * i + 1];
+        memmove((char *)k_cache + dst * block_bytes, (const char *)k_cache + src * block_bytes, (size_t)block_bytes);
+        memmove((char *)v_cache + dst * block_bytes, (const char *)v_cache + src * block_bytes, (size_t)block_bytes);
+    }
+    return 0;
+}
+
+/*
+ * pa_oracle_swap_blocks: for each pair i, block pairs[2i+1] of dst becomes a
+ * byte copy of block pairs[2i] of src (one pool; call once for K and once for
+ * V). src and dst may hold different numbers of blocks. Returns 0 or -1.
+ */
+int pa_oracle_swap_blocks(void *dst, const void *src, const int64_t *pairs, long num_pairs, long src_blocks,
+                          long dst_blocks, long block_bytes)
+{
+    for (long i = 0; i < num_pairs; ++i)
+        if (pairs[2 * i] < 0 || pairs[2 * i] >= src_blocks || pairs[2 * i + 1] < 0 || pairs[2 * i + 1] >= dst_blocks)
+            return -1;
+    for (long i = 0; i < num_pairs; ++i)
+        memcpy((char *)dst + pairs[2 * i + 1] * block_bytes, (const char *)src + pairs[2 * i] * block_bytes,
+               (size_t)block_bytes);
+    return 0;
+}

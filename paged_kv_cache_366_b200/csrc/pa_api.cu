@@ -10,6 +10,7 @@
 #include "pa_common.cuh"
 #include "decode.cuh"
 #include "prefill_sm100.cuh"
+#include "block_copy.cuh"
 #include "reshape_and_cache.cuh"
 
 namespace {
@@ -330,6 +331,61 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
     }
     return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                      max_context_len, scale, partition_tokens, scratch, need, shape, stream);
+}
+
+static int launch_copy(void *dst, const void *src, const int64_t *pairs, int64_t num_pairs, int64_t src_blocks,
+                       int64_t dst_blocks, int64_t block_bytes, cudaStream_t st) {
+    if (block_bytes <= 0 || block_bytes % 16 != 0 || block_bytes / 16 > (int64_t{1} << 30)) return PA_ERR_UNSUPPORTED;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    int64_t grid = num_pairs < int64_t{sms} * 8 ? num_pairs : int64_t{sms} * 8;
+    pa::copy_blocks_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(
+        static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), pairs, num_pairs, src_blocks, dst_blocks,
+        static_cast<int>(block_bytes / 16));
+    return check_launch();
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pairs, int64_t num_pairs,
+                   const pa_shape *shape, void *stream) {
+    int rc = check_shape(shape);
+    if (rc != PA_OK) return rc;
+    if (num_pairs < 0) return PA_ERR_INVALID_ARGUMENT;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !block_pairs) return PA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_pairs, 8)) return PA_ERR_ALIGNMENT;
+    const int64_t bb = int64_t{PA_BLOCK_SIZE} * shape->num_kv_heads * shape->head_dim * elem_bytes(shape);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_copy(k_cache, k_cache, block_pairs, num_pairs, shape->num_blocks, shape->num_blocks, bb, st);
+    if (rc != PA_OK) return rc;
+    return launch_copy(v_cache, v_cache, block_pairs, num_pairs, shape->num_blocks, shape->num_blocks, bb, st);
+}
+
+// Device address of memory a kernel may touch: device memory, or pinned host
+// memory through its mapping. Pageable host memory is refused.
+static int device_view(const void *p, void **dev) {
+    cudaPointerAttributes a;
+    const cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return PA_ERR_INVALID_ARGUMENT;
+    }
+    if (a.type == cudaMemoryTypeUnregistered || a.devicePointer == nullptr) return PA_ERR_INVALID_ARGUMENT;
+    *dev = a.devicePointer;
+    return PA_OK;
+}
+
+int pa_swap_blocks(void *dst, const void *src, const int64_t *block_pairs, int64_t num_pairs, int64_t src_blocks,
+                   int64_t dst_blocks, int64_t block_bytes, void *stream) {
+    if (num_pairs < 0 || src_blocks <= 0 || dst_blocks <= 0) return PA_ERR_INVALID_ARGUMENT;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst || !src || !block_pairs) return PA_ERR_INVALID_ARGUMENT;
+    void *d = nullptr, *s = nullptr, *pr = nullptr;
+    int rc = device_view(dst, &d);
+    if (rc == PA_OK) rc = device_view(src, &s);
+    if (rc == PA_OK) rc = device_view(block_pairs, &pr);
+    if (rc != PA_OK) return rc;
+    if (!aligned16(d) || !aligned16(s) || !aligned(pr, 8)) return PA_ERR_ALIGNMENT;
+    return launch_copy(d, s, static_cast<const int64_t *>(pr), num_pairs, src_blocks, dst_blocks, block_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int pa_get_status(uint32_t *status, void *stream) {

@@ -41,6 +41,7 @@ class PaShape(ctypes.Structure):
 EXPORTED = [
     "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
     "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version", "pa_decode_noalloc",
+    "pa_copy_blocks", "pa_swap_blocks",
 ]
 
 PA_ERR_SCRATCH_LIMIT = -7
@@ -63,6 +64,10 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_prefill_chunk.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, SP, P]
     lib.pa_decode_noalloc.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [P, P, P, I64, SP, P]
+    lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_swap_blocks.argtypes = [P, P, P, I64, I64, I64, I64, P]
+    lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
     lib.pa_get_status.restype = ctypes.c_int
     lib.pa_strerror.argtypes = [ctypes.c_int]
@@ -211,6 +216,34 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_
            lib.pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                 block_tables.shape[1], _ptr(cu_q_lens), _ptr(context_lens), B, int(max_q_len), T,
                                 float(scale), ctypes.byref(shape), _stream(stream)))
+
+
+def pa_copy_blocks(k_cache, v_cache, block_pairs, stream=None) -> None:
+    """Copy whole blocks inside the pool: block_pairs int64 [n, 2] of (src, dst), on the device."""
+    _same_dtype(k_cache, v_cache)
+    _int(block_pairs, torch.int64, "block_pairs")
+    shape = shape_of(k_cache, k_cache.shape[2])
+    _check("pa_copy_blocks", lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_pairs),
+                                                block_pairs.numel() // 2, ctypes.byref(shape), _stream(stream)))
+
+
+def _any_ptr(t: torch.Tensor):
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError("host tensors must be pinned")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_swap_blocks(dst, src, block_pairs, stream=None) -> None:
+    """Copy blocks of one pool between device and pinned host memory: block_pairs int64 [n, 2] of (src, dst)."""
+    if dst.dtype != src.dtype or dst.shape[1:] != src.shape[1:]:
+        raise ValueError("dst and src pools must have the same dtype and block shape")
+    _int(block_pairs, torch.int64, "block_pairs")
+    bb = src[0].numel() * src.element_size()
+    _check("pa_swap_blocks", lib.pa_swap_blocks(_any_ptr(dst), _any_ptr(src), _any_ptr(block_pairs),
+                                                block_pairs.numel() // 2, src.shape[0], dst.shape[0], bb,
+                                                _stream(stream)))
 
 
 def pa_get_status(stream=None) -> int:

@@ -380,3 +380,68 @@ def test_planted_mistakes_are_caught(mutation):
     finally:
         oracle.set_mutation(0)
     assert failures, "mutation %d passed every pin" % mutation
+
+
+# ---------------------------------------------------------------------------
+# Block copies (copy-on-write fork, swap out/in), pinned by the attention they preserve.
+
+def _fork_case(seed=181):
+    # two sequences sharing all three blocks of a 37-token prefix; each appends one token
+    return W.make_case("fork", seed, context_lens=[37, 37], q_lens=[0, 0], num_heads=8, num_kv_heads=2,
+                       head_dim=64, dtype="f32", shared_prefix_blocks=2, keep_logical=True, table_slack=1)
+
+
+def test_copy_on_write_fork_keeps_sequences_apart():
+    """After copying the shared last block for sequence 1 and writing each sequence's
+    next token into its own last block, each sequence attends to its own token."""
+    case = _fork_case()
+    bt = case.block_tables.copy()
+    bt[1, :3] = bt[0, :3]  # sequence 1 shares all of sequence 0's blocks, the partial last one too
+    kc, vc = case.k_cache.copy(), case.v_cache.copy()
+    free = np.setdiff1d(np.arange(case.num_blocks), bt[bt >= 0])
+    new_blk = int(free[0])
+    kc, vc = oracle.copy_blocks(kc, vc, [[bt[0, 2], new_blk]])
+    bt[1, 2] = new_blk
+    rng = np.random.default_rng(3)
+    k_tok = rng.uniform(-1, 1, (2, 2, 64)).astype(np.float32)
+    v_tok = rng.uniform(-1, 1, (2, 2, 64)).astype(np.float32)
+    slots = np.array([oracle.slot_of(bt[0], 37), oracle.slot_of(bt[1], 37)], np.int64)
+    kc, vc = oracle.reshape_and_cache(k_tok, v_tok, kc, vc, slots)
+    lens = np.array([38, 38], np.int32)
+    q = rng.uniform(-1, 1, (2, 8, 64)).astype(np.float32)
+    out = oracle.decode(q, kc, vc, bt, lens, 0.3)
+    # reference: each sequence's own contiguous history + its own token, by library attention
+    for b in range(2):
+        K = np.concatenate([widen(case.logical_k[0][:37]), k_tok[b][None]], 0)
+        V = np.concatenate([widen(case.logical_v[0][:37]), v_tok[b][None]], 0)
+        o = F.scaled_dot_product_attention(torch.from_numpy(q[b].astype(np.float64))[None, :, None, :],
+                                           torch.from_numpy(K).permute(1, 0, 2)[None],
+                                           torch.from_numpy(V).permute(1, 0, 2)[None], scale=0.3, enable_gqa=True)
+        assert np.abs(out[b] - o[0, :, 0, :].numpy()).max() <= TOL
+
+
+def test_swap_out_and_in_preserves_attention():
+    case = small_decode_case(191, dtype="bf16", D=128)
+    kc, vc = written(case)
+    base = oracle.decode(case.q, kc, vc, case.block_tables, case.context_lens, case.scale)
+    used = np.unique(case.block_tables[case.block_tables >= 0])
+    host_k = np.zeros((len(used) + 3,) + kc.shape[1:], kc.dtype)
+    host_v = np.zeros_like(host_k)
+    out_pairs = np.stack([used, np.arange(len(used)) + 3], 1)
+    host_k = oracle.swap_blocks(host_k, kc, out_pairs)
+    host_v = oracle.swap_blocks(host_v, vc, out_pairs)
+    # bring them back to a permuted set of device blocks and rewrite the tables
+    new_ids = np.random.default_rng(9).permutation(case.num_blocks)[:len(used)]
+    in_pairs = np.stack([np.arange(len(used)) + 3, new_ids], 1)
+    kc2 = oracle.swap_blocks(np.full_like(kc, 0), host_k, in_pairs)
+    vc2 = oracle.swap_blocks(np.full_like(vc, 0), host_v, in_pairs)
+    remap = dict(zip(used.tolist(), new_ids.tolist()))
+    bt2 = np.vectorize(lambda x: remap.get(int(x), -1))(case.block_tables).astype(np.int32)
+    moved = oracle.decode(case.q, kc2, vc2, bt2, case.context_lens, case.scale)
+    assert np.array_equal(base, moved)
+
+
+def test_block_copy_rejects_indices_outside_the_pool():
+    case = small_decode_case(201)
+    with pytest.raises(oracle.OracleError):
+        oracle.copy_blocks(case.k_cache, case.v_cache, [[0, case.num_blocks]])
