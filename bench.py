@@ -48,7 +48,8 @@ FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
 WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny",
-             "copy_blocks", "swap_blocks"]
+             "copy_blocks", "swap_blocks", "decode_batch_fp8"]
+FP8_K_SCALE, FP8_V_SCALE = 0.02, 1.0 / 48.0
 BLOCK_WORKLOADS = ("copy_blocks", "swap_blocks")
 BLOCK_PAIRS = 2048
 
@@ -67,13 +68,14 @@ def split_seqs(case):
     return dec, pre
 
 
-def step_bytes(case, dec, pre):
-    """Algorithmic bytes of one step, by part."""
+def step_bytes(case, dec, pre, kv_elem=None):
+    """Algorithmic bytes of one step, by part (kv_elem: bytes per cache element, default the case's)."""
     E, H, Hk, D = case.elem_bytes, case.num_heads, case.num_kv_heads, case.head_dim
+    KE = E if kv_elem is None else kv_elem
     ctx = case.context_lens.astype(np.int64)
     T = case.num_tokens
-    write = T * Hk * D * E * 2 * 2 + T * 8
-    kv_dec = int(ctx[dec].sum()) * Hk * D * E * 2
+    write = T * Hk * D * (E + KE) * 2 + T * 8
+    kv_dec = int(ctx[dec].sum()) * Hk * D * KE * 2
     tables_dec = int(((ctx[dec] + 15) // 16).sum()) * 4 + 4 * len(dec)
     decode = kv_dec + len(dec) * H * D * E * 2 + tables_dec
     prefill = 0
@@ -313,6 +315,8 @@ def run_reference(args):
 # GPU arm
 
 def make_workload(name):
+    if name == "decode_batch_fp8":
+        return W.decode_batch()
     if name not in W.CONFIGS:
         raise SystemExit("unknown workload %s (one of %s)" % (name, ", ".join(WORKLOADS)))
     return W.CONFIGS[name]()
@@ -342,13 +346,25 @@ def run_ours(args):
 
     case = make_workload(args.workload)
     dec, pre = split_seqs(case)
-    nbytes = step_bytes(case, dec, pre)
+    fp8 = args.workload == "decode_batch_fp8"
+    ks, vs = (FP8_K_SCALE, FP8_V_SCALE) if fp8 else (0.0, 0.0)
+    nbytes = step_bytes(case, dec, pre, 1 if fp8 else None)
 
     k_cache, v_cache = dev(case.k_cache), dev(case.v_cache)
+    if fp8:  # quantize the whole pool with the library's own FP8 write
+        NB, bs, Hk, D = case.k_cache.shape
+        kc8 = torch.empty(tuple(k_cache.shape), dtype=torch.uint8, device="cuda")
+        vc8 = torch.empty_like(kc8)
+        every_slot = torch.arange(NB * bs, dtype=torch.int64, device="cuda")
+        pa.pa_reshape_and_cache(k_cache.view(NB * bs, Hk, D), v_cache.view(NB * bs, Hk, D), kc8, vc8, every_slot,
+                                k_scale=ks, v_scale=vs)
+        torch.cuda.synchronize()
+        del k_cache, v_cache, every_slot
+        k_cache, v_cache = kc8, vc8
     k_new, v_new, q = dev(case.k_new), dev(case.v_new), dev(case.q)
     slots = dev(case.slot_mapping)
     tables, lens, cu = dev(case.block_tables), dev(case.context_lens), dev(case.cu_q_lens)
-    shape = pa.shape_of(k_cache, case.num_heads)
+    shape = pa.shape_of(k_cache, case.num_heads, ks, vs)
 
     d0, d1 = (int(dec[0]), int(dec[-1]) + 1) if len(dec) else (0, 0)
     dec_rows = torch.from_numpy(np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)).cuda()
@@ -370,10 +386,11 @@ def run_ours(args):
     stream = torch.cuda.Stream()
 
     def do_write():
-        pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots)
+        pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, k_scale=ks, v_scale=vs)
 
     def do_decode():
-        pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws)
+        pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws,
+                     k_scale=ks, v_scale=vs)
 
     def do_prefill():
         pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
@@ -478,7 +495,7 @@ def run_ours(args):
     if len(dec) and not len(pre):
         hk_cache = k_cache  # the pool is device-resident state
         step = DecodeStep(hk_cache, v_cache, case.num_heads, len(dec), case.max_blocks_per_seq, max_ctx,
-                          case.scale)
+                          case.scale, k_scale=ks, v_scale=vs)
 
         def pinned(a):
             t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16
@@ -487,6 +504,7 @@ def run_ours(args):
             return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
         rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)
         h_out = torch.empty(tuple(q_dec.shape), dtype=torch.int16 if case.dtype == "bf16" else torch.float32)
+        assert not fp8 or case.dtype == "bf16"
         h_out = h_out.pin_memory()
         if case.dtype == "bf16":
             h_out = h_out.view(torch.bfloat16)
@@ -534,6 +552,8 @@ def run_ours(args):
         cpu.pop("seconds", None)
     parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
+    if fp8:
+        config.update({"workload": "decode_batch_fp8", "kv_dtype": "fp8_e4m3", "k_scale": ks, "v_scale": vs})
     config.update({"l2": "flushed before every step, outside the events: 256 MiB memset, then a 256 MiB read "
                          "so the memset's write-back is not charged to the step",
                    "timing": "one CUDA graph replay per step between CUDA events on the launching stream; "

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 1
+#define PA_ABI_VERSION 2
 #define PA_BLOCK_SIZE 16
 
 typedef enum {
@@ -86,7 +86,20 @@ typedef struct {
     int32_t head_dim;     /* D: 64 or 128 */
     int32_t block_size;   /* tokens per block: must be 16 */
     int64_t num_blocks;   /* NB, blocks in the pool */
-    int32_t dtype;        /* pa_dtype */
+    int32_t dtype;        /* pa_dtype of q, out and the new tokens' k, v */
+    /*
+     * 0: the caches hold `dtype`. 1: they hold FP8 E4M3 codes, one byte per
+     * element (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+     * infinities, largest finite 448). A cached value means code * k_scale
+     * (keys) or code * v_scale (values). The write quantizes
+     * fp32(x) * fp32(1 / scale) to the nearest code (ties to even, saturating
+     * at +-448). FP8 caches need dtype = PA_DTYPE_BF16; pa_prefill_chunk does
+     * not take them. The pages name FP8 only for weights ("vLLM and
+     * PagedAttention" §5); an FP8 cache halves the bytes decode reads.
+     */
+    int32_t kv_fp8;
+    float k_scale; /* > 0 when kv_fp8; ignored otherwise */
+    float v_scale; /* > 0 when kv_fp8; ignored otherwise */
 } pa_shape;
 
 /*

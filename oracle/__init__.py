@@ -21,7 +21,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-F32, BF16 = 0, 1
+F32, BF16, FP8_E4M3 = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +58,14 @@ def _load():
             lib.pa_oracle_copy_blocks.restype = I
             lib.pa_oracle_swap_blocks.argtypes = [P, P, P, L, L, L, L]
             lib.pa_oracle_swap_blocks.restype = I
+            lib.pa_oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.pa_oracle_e4m3_decode.restype = D
+            lib.pa_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.pa_oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.pa_oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, L, L, L, ctypes.c_float, ctypes.c_float]
+            lib.pa_oracle_reshape_and_cache_fp8.restype = L
+            lib.pa_oracle_decode_fp8.argtypes = [P, P, I, P, P, D, D, P, I, P, I, I, I, I, I, L, D, I]
+            lib.pa_oracle_decode_fp8.restype = I
             lib.pa_oracle_set_mutation.argtypes = [I]
             lib.pa_oracle_set_mutation.restype = None
             lib.pa_oracle_get_mutation.argtypes = []
@@ -208,3 +216,48 @@ def swap_blocks(dst, src, pairs):
     if rc:
         raise OracleError("block index outside a pool")
     return d
+
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().pa_oracle_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(x: float) -> int:
+    """Nearest E4M3 code of a float32 value (ties to even, saturating at 448)."""
+    return int(_load().pa_oracle_e4m3_encode(float(np.float32(x))))
+
+
+def reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_inv_scale: float, v_inv_scale: float):
+    """Quantize bf16 rows (uint16 bits) into copies of the uint8 E4M3 caches at their slots."""
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    kc = np.array(k_cache, copy=True, order="C")
+    vc = np.array(v_cache, copy=True, order="C")
+    assert kc.dtype == np.uint8
+    sm = _c(slot_mapping, np.int64)
+    NB, bs, Hk, D = kc.shape
+    n = _load().pa_oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), _ptr(kc), _ptr(vc), _ptr(sm), sm.shape[0], NB * bs,
+                                                Hk * D, float(np.float32(k_inv_scale)), float(np.float32(v_inv_scale)))
+    if n < 0:
+        raise OracleError("slot outside the pool")
+    return kc, vc
+
+
+def decode_fp8(q, k_cache, v_cache, k_scale: float, v_scale: float, block_tables, context_lens, scale: float,
+               num_threads: int = 0):
+    """Decode over E4M3 caches (uint8 codes): K, V = code value times k_scale, v_scale."""
+    q = _c(q)
+    k_cache = _c(k_cache, np.uint8)
+    v_cache = _c(v_cache, np.uint8)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    B, H, D = q.shape
+    NB, bs, Hk, D2 = k_cache.shape
+    assert D == D2
+    out = np.zeros((B, H, D), np.float64)
+    rc = _load().pa_oracle_decode_fp8(_ptr(out), _ptr(q), _dtype_code(q), _ptr(k_cache), _ptr(v_cache),
+                                      float(k_scale), float(v_scale), _ptr(bt), bt.shape[1], _ptr(cl), B, H, Hk, D,
+                                      bs, NB, float(scale), int(num_threads))
+    if rc:
+        raise OracleError("decode failed (%d)" % rc)
+    return out

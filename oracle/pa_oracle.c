@@ -47,7 +47,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_FP8_E4M3 = 2 };
 
 enum {
     MUT_NONE = 0,
@@ -68,8 +68,63 @@ static int g_mutation = MUT_NONE;
 void pa_oracle_set_mutation(int m) { g_mutation = m; }
 int pa_oracle_get_mutation(void) { return g_mutation; }
 
+/*
+ * FP8 E4M3 (the "fn" variant: 1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no infinities, S.1111.111 is NaN, largest finite 448), written from
+ * the format's definition. Codes 0x01..0x07 are subnormals k * 2^-9.
+ */
+double pa_oracle_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+    double v;
+    if (e == 0xF && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Round a float to E4M3: nearest, ties to even; finite values past 448 saturate to 448. */
+uint8_t pa_oracle_e4m3_encode(float f)
+{
+    if (isnan(f))
+        return 0x7F;
+    uint8_t sign = signbit(f) ? 0x80 : 0;
+    double a = fabs((double)f);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    /* every representable magnitude is a multiple of its binade's quantum */
+    int e;
+    frexp(a, &e); /* a = f * 2^e with f in [0.5, 1): binade 2^(e-1) */
+    int be = e - 1;
+    if (be < -6)
+        be = -6; /* subnormals share the quantum of the lowest normal binade */
+    double q = ldexp(1.0, be - 3);
+    double n = a / q; /* exact: q is a power of two */
+    double r = floor(n);
+    double frac = n - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) == 1.0))
+        r += 1.0;
+    double v = r * q; /* the rounded magnitude */
+    if (v >= 448.0)
+        return sign | 0x7E;
+    if (v == 0.0)
+        return sign;
+    if (v < ldexp(1.0, -6))
+        return sign | (uint8_t)(v / ldexp(1.0, -9));
+    int ve;
+    double vf = frexp(v, &ve); /* v = vf * 2^ve, vf in [0.5, 1) */
+    int exp_field = ve - 1 + 7;
+    int mant = (int)((vf * 2.0 - 1.0) * 8.0);
+    return sign | (uint8_t)(exp_field << 3) | (uint8_t)mant;
+}
+
 static double load_elem(const void *base, long idx, int dtype)
 {
+    if (dtype == ORACLE_FP8_E4M3)
+        return pa_oracle_e4m3_decode(((const uint8_t *)base)[idx]);
     if (dtype == ORACLE_BF16) {
         uint32_t u = (uint32_t)((const uint16_t *)base)[idx] << 16;
         float f;
@@ -385,4 +440,86 @@ int pa_oracle_swap_blocks(void *dst, const void *src, const int64_t *pairs, long
         memcpy((char *)dst + pairs[2 * i + 1] * block_bytes, (const char *)src + pairs[2 * i] * block_bytes,
                (size_t)block_bytes);
     return 0;
+}
+
+/*
+ * FP8 cache write: the new tokens' K/V rows (bf16 bits) are quantized to E4M3
+ * with the same fp32 steps the kernel takes: x -> fp32, times inv_scale in
+ * fp32 (one IEEE multiply), then E4M3 rounding. Dequantized value =
+ * e4m3(code) * scale with scale = 1 / inv_scale. Returns tokens written or -1.
+ */
+long pa_oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v, uint8_t *k_cache, uint8_t *v_cache,
+                                     const int64_t *slot_mapping, long num_tokens, long num_slots, long row_elems,
+                                     float k_inv_scale, float v_inv_scale)
+{
+    for (long t = 0; t < num_tokens; ++t)
+        if (slot_mapping[t] >= num_slots)
+            return -1;
+    long written = 0;
+    for (long t = 0; t < num_tokens; ++t) {
+        long s = slot_mapping[t];
+        if (s < 0)
+            continue;
+        for (long i = 0; i < row_elems; ++i) {
+            uint32_t ku = (uint32_t)k[t * row_elems + i] << 16, vu = (uint32_t)v[t * row_elems + i] << 16;
+            float kf, vf;
+            memcpy(&kf, &ku, 4);
+            memcpy(&vf, &vu, 4);
+            volatile float kq = kf * k_inv_scale, vq = vf * v_inv_scale; /* fp32 products */
+            k_cache[s * row_elems + i] = pa_oracle_e4m3_encode(kq);
+            v_cache[s * row_elems + i] = pa_oracle_e4m3_encode(vq);
+        }
+        ++written;
+    }
+    return written;
+}
+
+/*
+ * Decode over an FP8 E4M3 cache: K = e4m3(code) * k_scale, V = e4m3(code) *
+ * v_scale, q and out as q_dtype. Otherwise identical to pa_oracle_decode.
+ */
+int pa_oracle_decode_fp8(double *out, const void *q, int q_dtype, const uint8_t *k_cache, const uint8_t *v_cache,
+                         double k_scale, double v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                         int block_size, long num_blocks, double scale, int num_threads)
+{
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
+        return -2;
+    int nt = set_threads(num_threads);
+    int status = 0;
+    long units = (long)num_seqs * num_kv_heads;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (long u = 0; u < units; ++u) {
+        int b = (int)(u / num_kv_heads), hk = (int)(u % num_kv_heads);
+        long c = context_lens[b];
+        double *Kc = malloc(sizeof(double) * (size_t)(c > 0 ? c : 1) * head_dim);
+        double *Vc = malloc(sizeof(double) * (size_t)(c > 0 ? c : 1) * head_dim);
+        double *s = malloc(sizeof(double) * (size_t)(c > 0 ? c : 1));
+        double *qv = malloc(sizeof(double) * (size_t)head_dim);
+        int rc = (c < 0) ? -2 : pa_oracle_gather(Kc, Vc, k_cache, v_cache, ORACLE_FP8_E4M3, block_tables,
+                                                  max_blocks_per_seq, b, c, num_kv_heads, hk, head_dim,
+                                                  block_size, num_blocks);
+        if (rc) {
+#pragma omp critical
+            status = rc;
+        } else {
+            for (long i = 0; i < c * head_dim; ++i) {
+                Kc[i] *= k_scale;
+                Vc[i] *= v_scale;
+            }
+            for (int h = 0; h < num_heads; ++h) {
+                if (kv_head_of(h, num_heads, num_kv_heads) != hk)
+                    continue;
+                long qbase = ((long)b * num_heads + h) * head_dim;
+                for (int d = 0; d < head_dim; ++d)
+                    qv[d] = load_elem(q, qbase + d, q_dtype);
+                attend(out + qbase, qv, Kc, Vc, readable_tokens(c, block_size), head_dim, scale, s);
+            }
+        }
+        free(Kc);
+        free(Vc);
+        free(s);
+        free(qv);
+    }
+    return status;
 }

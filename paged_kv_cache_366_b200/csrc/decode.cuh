@@ -46,7 +46,7 @@ template <typename T, int D, int G>
 struct DecodeCfg {
     static constexpr int E = sizeof(T);
     static constexpr int R = D * E;                        // bytes of one token row of one KV head
-    static constexpr int CH = G >= 8 ? 1 : 2;              // 16-byte chunks a lane owns per row
+    static constexpr int CH = (G >= 8 || E == 1) ? 1 : 2;  // 16-byte chunks a lane owns per row
     static constexpr int L = R / (16 * CH);                // lanes covering one row
     static constexpr int RS = 32 / L;                      // rows per warp step
     static constexpr int STEPS = kBlockSize / RS;          // steps per block
@@ -121,14 +121,17 @@ struct DecodeParams {
     int max_context_len;
     int part_tokens;
     int max_parts;
-    float scale_log2;  // softmax scale * log2(e)
+    float scale_log2;  // softmax scale * log2(e) (times k_scale for an FP8 cache)
+    float v_scale;     // 1, or the FP8 value scale
 };
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS)
+// Tq: element type of q and out. Tc: element type of the caches (the same, or
+// FP8 E4M3 codes with bf16 q/out).
+template <typename Tq, typename Tc, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCKS)
     decode_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
-    using C = DecodeCfg<T, D, G>;
+    using C = DecodeCfg<Tc, D, G>;
     // Grid (KV head, sequence, partition): every unit's first partition launches
     // before any second one, so full partitions run first and the short last
     // partitions (or empty CTAs) form the tail.
@@ -136,6 +139,9 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
     // Launched as a programmatic dependent (its launch overlaps the previous
     // kernel, e.g. the cache write): wait for that kernel before reading any input.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The merge kernel may be scheduled as soon as every CTA of this grid has
+    // started; it still waits for this grid to finish before reading partials.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
     const int c = clamp_context(__ldg(prm.context_lens + b), cap, p == 0 && hk == 0 && threadIdx.x == 0);
     const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
@@ -195,14 +201,20 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
     constexpr int VP = C::VE / 2;   // packed pairs per 16-byte chunk
     f32x2 q2[G][P2];
     {
-        const T *qb = static_cast<const T *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
+        // the lane's dims in q: the same VE-element chunks as in the cache row
+        constexpr int QV = C::VE * static_cast<int>(sizeof(Tq)) / 16;  // 16-byte q loads per chunk
+        constexpr int QP = Widen<Tq>::N / 2;                            // pairs per q load
+        const Tq *qb = static_cast<const Tq *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
         const f32x2 sc = pack2(prm.scale_log2, prm.scale_log2);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + (ch * C::L + j) * C::VE));
-                Widen<T>::apply2(raw, &q2[g][ch * VP]);
+#pragma unroll
+                for (int u = 0; u < QV; ++u) {
+                    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + (ch * C::L + j) * C::VE) + u);
+                    Widen<Tq>::apply2(raw, &q2[g][ch * VP + u * QP]);
+                }
 #pragma unroll
                 for (int e = 0; e < VP; ++e) mul2(q2[g][ch * VP + e], sc);
             }
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(kb + row * C::R + (ch * C::L + j) * 16);
-                Widen<T>::apply2(raw, &k2[ch * VP]);
+                Widen<Tc>::apply2(raw, &k2[ch * VP]);
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -324,7 +336,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(vb + t * C::R + (ch * C::L + j) * 16);
-                Widen<T>::apply2(raw, &v2[ch * VP]);
+                Widen<Tc>::apply2(raw, &v2[ch * VP]);
             }
             if (t < n_valid) {
 #pragma unroll
@@ -388,9 +400,10 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
                 Lsum += wt * red_l[w * G + g];
             }
         }
+        O *= prm.v_scale;
         const int h = hk * G + g;
         if (parts == 1) {
-            T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
+            Tq *out = static_cast<Tq *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
             store_out(out, Lsum > 0.f ? O / Lsum : 0.f);
         } else {
             const size_t pi = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts + p;
@@ -401,8 +414,6 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
             }
         }
     }
-    // let the merge kernel (launched as a programmatic dependent) get scheduled
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the partitions of every sequence that has more than one:
@@ -412,7 +423,8 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<T, D, G>::MIN_BLOCKS
 // (griddepcontrol.wait) before reading the partials.
 template <typename T>
 __global__ void decode_reduce_kernel(const DecodeParams prm, int D) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // context_lens was written before decode_kernel ran (decode_kernel waited for
+    // it), so it may be read before waiting for decode_kernel's partials.
     const int hk = blockIdx.x, b = blockIdx.y;
     const int G = prm.num_heads / prm.num_kv_heads;
     const int g = threadIdx.x / D, d = threadIdx.x % D;
@@ -420,6 +432,7 @@ __global__ void decode_reduce_kernel(const DecodeParams prm, int D) {
     const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
     const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
     if (parts == 1 || g >= G) return;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int h = hk * G + g;
     const size_t base = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts;
     // one pass with a running max: the loads of up to 8 partitions go out together

@@ -54,10 +54,17 @@ int check_shape(const pa_shape *s) {
     const int g = s->num_heads / s->num_kv_heads;
     if (g != 1 && g != 2 && g != 4 && g != 8) return PA_ERR_UNSUPPORTED;
     if (s->num_blocks >= (int64_t{1} << 31) / PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;  // rows fit in int32 math
+    if (s->kv_fp8 != 0 && s->kv_fp8 != 1) return PA_ERR_INVALID_ARGUMENT;
+    if (s->kv_fp8) {
+        if (s->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+        if (!(s->k_scale > 0.f) || !(s->v_scale > 0.f) || !std::isfinite(s->k_scale) || !std::isfinite(s->v_scale))
+            return PA_ERR_INVALID_ARGUMENT;
+    }
     return PA_OK;
 }
 
 int elem_bytes(const pa_shape *s) { return s->dtype == PA_DTYPE_BF16 ? 2 : 4; }
+int cache_elem_bytes(const pa_shape *s) { return s->kv_fp8 ? 1 : elem_bytes(s); }
 
 // Tokens per split-context partition. A context of at most one partition is
 // handled by the single pass alone (no workspace, no reduce kernel).
@@ -112,17 +119,17 @@ int allow_smem(K kernel, int bytes, std::atomic<uint64_t> &done) {
     return PA_OK;
 }
 
-template <typename T, int D, int G>
+template <typename Tq, typename Tc, int D, int G>
 int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
-    using C = pa::DecodeCfg<T, D, G>;
+    using C = pa::DecodeCfg<Tc, D, G>;
     static std::atomic<uint64_t> smem_done{0};
-    int arc = allow_smem(pa::decode_kernel<T, D, G>, C::SMEM, smem_done);
+    int arc = allow_smem(pa::decode_kernel<Tq, Tc, D, G>, C::SMEM, smem_done);
     if (arc != PA_OK) return arc;
     CUtensorMap tm_k{}, tm_v{};
     const uint64_t rows = static_cast<uint64_t>(prm.num_blocks) * pa::kBlockSize;
-    if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(T), D, 1, pa::kBlockSize,
+    if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(T), D, 1, pa::kBlockSize,
+        !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
         return PA_ERR_UNSUPPORTED;
     // Both kernels are programmatic dependent launches: each starts launching
@@ -138,23 +145,23 @@ int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<T, D, G>, prm, tm_k, tm_v);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
     if (e != cudaSuccess) return cuda_fail(e);
     if (prm.max_parts == 1) return PA_OK;
     cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
     cfg.blockDim = dim3(G * D);
     cfg.dynamicSmemBytes = 0;
-    e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<T>, prm, D);
+    e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
-template <typename T, int D>
+template <typename Tq, typename Tc, int D>
 int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
     switch (g) {
-        case 1: return launch_decode<T, D, 1>(prm, num_seqs, st);
-        case 2: return launch_decode<T, D, 2>(prm, num_seqs, st);
-        case 4: return launch_decode<T, D, 4>(prm, num_seqs, st);
-        case 8: return launch_decode<T, D, 8>(prm, num_seqs, st);
+        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st);
+        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st);
+        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st);
+        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -190,7 +197,7 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
     if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARGUMENT;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(slot_mapping, 8))
         return PA_ERR_ALIGNMENT;
-    const int row_bytes = shape->num_kv_heads * shape->head_dim * elem_bytes(shape);
+    const int row_bytes = shape->num_kv_heads * shape->head_dim * elem_bytes(shape);  // one input row
     if (row_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
     const int row_vecs = row_bytes / 16;
     const int64_t total = num_tokens * row_vecs;
@@ -198,7 +205,15 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
     int64_t blocks = (total + threads - 1) / threads;
     const int sms = sm_count() > 0 ? sm_count() : 148;
     if (blocks > int64_t{sms} * 16) blocks = int64_t{sms} * 16;
-    pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (shape->kv_fp8) {
+        pa::reshape_and_cache_fp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint2 *>(k_cache),
+            static_cast<uint2 *>(v_cache), slot_mapping, num_tokens, shape->num_blocks * PA_BLOCK_SIZE, row_vecs,
+            1.0f / shape->k_scale, 1.0f / shape->v_scale);
+        return check_launch();
+    }
+    pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
         static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
         static_cast<uint4 *>(v_cache), slot_mapping, num_tokens, shape->num_blocks * PA_BLOCK_SIZE, row_vecs);
     return check_launch();
@@ -255,14 +270,23 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     prm.part_tokens = g.part_tokens;
     prm.max_parts = g.max_parts;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.v_scale = 1.f;
+    if (shape->kv_fp8) {
+        prm.scale_log2 *= shape->k_scale;
+        prm.v_scale = shape->v_scale;
+    }
     const int G = shape->num_heads / shape->num_kv_heads;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (shape->dtype == PA_DTYPE_BF16) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, 128>(G, prm, num_seqs, st)
-                                      : dispatch_g<__nv_bfloat16, 64>(G, prm, num_seqs, st);
+    if (shape->kv_fp8) {
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st)
+                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st);
     }
-    return shape->head_dim == 128 ? dispatch_g<float, 128>(G, prm, num_seqs, st)
-                                  : dispatch_g<float, 64>(G, prm, num_seqs, st);
+    if (shape->dtype == PA_DTYPE_BF16) {
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st)
+                                      : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st);
+    }
+    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st)
+                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -271,7 +295,7 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
                      void *stream) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
-    if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128 || shape->kv_fp8) return PA_ERR_UNSUPPORTED;
     if (num_seqs < 0 || max_q_len < 0 || num_q_tokens < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
     if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens)
@@ -352,7 +376,7 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pairs, int
     if (num_pairs == 0) return PA_OK;
     if (!k_cache || !v_cache || !block_pairs) return PA_ERR_INVALID_ARGUMENT;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_pairs, 8)) return PA_ERR_ALIGNMENT;
-    const int64_t bb = int64_t{PA_BLOCK_SIZE} * shape->num_kv_heads * shape->head_dim * elem_bytes(shape);
+    const int64_t bb = int64_t{PA_BLOCK_SIZE} * shape->num_kv_heads * shape->head_dim * cache_elem_bytes(shape);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = launch_copy(k_cache, k_cache, block_pairs, num_pairs, shape->num_blocks, shape->num_blocks, bb, st);
     if (rc != PA_OK) return rc;

@@ -141,9 +141,57 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// Widen 16 bytes of storage to fp32: 8 bf16 or 4 fp32 values.
+// One FP8 E4M3 code (cache storage type).
+struct fp8e4m3 {
+    uint8_t bits;
+};
+
+// Two E4M3 codes (low byte = element 0) to two fp32 values, exactly.
+__device__ __forceinline__ f32x2 e4m3x2_to_f32x2(uint32_t two_codes) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 c;\n\t"
+        "cvt.u16.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(two_codes));
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h2));
+    return pack2(lo, hi);
+}
+
+// Two fp32 values to two E4M3 codes in the low 16 bits (low byte = x0):
+// nearest, ties to even, saturating at +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x0, float x1) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 c;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c, %2, %1;\n\t"
+        "cvt.u32.u16 %0, c;\n\t}"
+        : "=r"(r)
+        : "f"(x0), "f"(x1));
+    return r;
+}
+
+// Widen 16 bytes of storage to fp32: 16 fp8, 8 bf16 or 4 fp32 values.
 template <typename T>
 struct Widen;
+
+template <>
+struct Widen<fp8e4m3> {
+    static constexpr int N = 16;
+    __device__ __forceinline__ static void apply2(const uint4 &r, f32x2 *f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = e4m3x2_to_f32x2(w[i] & 0xffffu);
+            f[2 * i + 1] = e4m3x2_to_f32x2(w[i] >> 16);
+        }
+    }
+};
 
 template <>
 struct Widen<__nv_bfloat16> {

@@ -34,7 +34,9 @@ inline bool encode_3d(CUtensorMap *m, const void *base, uint64_t n0, uint64_t n1
                       uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
-    const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType dt = elem == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const cuuint64_t dims[3] = {n0, n1, n2};
     const cuuint64_t strides[2] = {n0 * elem, n1 * n0 * elem};
     const cuuint32_t box[3] = {b0, b1, b2};

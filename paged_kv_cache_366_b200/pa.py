@@ -35,6 +35,9 @@ class PaShape(ctypes.Structure):
         ("block_size", ctypes.c_int32),
         ("num_blocks", ctypes.c_int64),
         ("dtype", ctypes.c_int32),
+        ("kv_fp8", ctypes.c_int32),
+        ("k_scale", ctypes.c_float),
+        ("v_scale", ctypes.c_float),
     ]
 
 
@@ -120,13 +123,30 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError("dtype must be bfloat16 or float32, got %s" % dt)
 
 
-def shape_of(k_cache: torch.Tensor, num_heads: int) -> PaShape:
-    """pa_shape of a pool [NB, 16, Hk, D] read by `num_heads` query heads."""
+def shape_of(k_cache: torch.Tensor, num_heads: int, k_scale: float = 0.0, v_scale: float = 0.0) -> PaShape:
+    """pa_shape of a pool [NB, 16, Hk, D] read by `num_heads` query heads.
+
+    A uint8 pool holds FP8 E4M3 codes (values code * k_scale / code * v_scale)
+    next to bf16 q/out and new tokens.
+    """
     if k_cache.dim() != 4:
         raise ValueError("k_cache must be [num_blocks, block_size, num_kv_heads, head_dim]")
     nb, bs, hk, d = k_cache.shape
+    fp8 = k_cache.dtype == torch.uint8
     return PaShape(num_heads=int(num_heads), num_kv_heads=int(hk), head_dim=int(d), block_size=int(bs),
-                   num_blocks=int(nb), dtype=_dtype_code(k_cache.dtype))
+                   num_blocks=int(nb), dtype=PA_DTYPE_BF16 if fp8 else _dtype_code(k_cache.dtype),
+                   kv_fp8=1 if fp8 else 0, k_scale=float(k_scale), v_scale=float(v_scale))
+
+
+def _same_dtype_kv(q_like, caches):
+    """q/out/new tokens share one dtype; caches share it or are uint8 FP8 codes with bf16 elsewhere."""
+    _same_dtype(*q_like)
+    _same_dtype(*caches)
+    if caches[0].dtype == torch.uint8:
+        if q_like[0].dtype != torch.bfloat16:
+            raise ValueError("an FP8 cache goes with bf16 q, out and new tokens")
+    elif caches[0].dtype != q_like[0].dtype:
+        raise ValueError("q/out/k/v and the caches must share one dtype")
 
 
 def _same_dtype(*ts):
@@ -140,11 +160,12 @@ def _int(t: torch.Tensor, dt: torch.dtype, name: str):
         raise ValueError("%s must be %s" % (name, dt))
 
 
-def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> None:
-    """Write each new token's K/V row into its slot of the pool (bit-exact copy)."""
-    _same_dtype(k, v, k_cache, v_cache)
+def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None, k_scale: float = 0.0,
+                         v_scale: float = 0.0) -> None:
+    """Write each new token's K/V row into its slot of the pool (bit-exact copy, or FP8 quantization)."""
+    _same_dtype_kv((k, v), (k_cache, v_cache))
     _int(slot_mapping, torch.int64, "slot_mapping")
-    shape = shape_of(k_cache, k_cache.shape[2])
+    shape = shape_of(k_cache, k_cache.shape[2], k_scale, v_scale)
     if k.shape[1:] != k_cache.shape[2:] or v.shape != k.shape or slot_mapping.shape[0] != k.shape[0]:
         raise ValueError("k, v must be [T, Hk, D] matching the cache; slot_mapping [T]")
     _check("pa_reshape_and_cache",
@@ -161,15 +182,16 @@ def pa_decode_workspace_bytes(num_seqs: int, max_context_len: int, partition_tok
 
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
-              partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+              partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+              k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """Decode attention of one query token per sequence over its paged context."""
-    _same_dtype(out, q, k_cache, v_cache)
+    _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(context_lens, torch.int32, "context_lens")
     B, H, D = q.shape
     if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
-    shape = shape_of(k_cache, H)
+    shape = shape_of(k_cache, H, k_scale, v_scale)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("pa_decode",
            lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
@@ -203,7 +225,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_
 def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
                      scale: float, stream=None) -> None:
     """Causal attention of query chunks at their context offsets (bf16, D=128)."""
-    _same_dtype(out, q, k_cache, v_cache)
+    _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(cu_q_lens, torch.int32, "cu_q_lens")
     _int(context_lens, torch.int32, "context_lens")
@@ -222,7 +244,7 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, stream=None) -> None:
     """Copy whole blocks inside the pool: block_pairs int64 [n, 2] of (src, dst), on the device."""
     _same_dtype(k_cache, v_cache)
     _int(block_pairs, torch.int64, "block_pairs")
-    shape = shape_of(k_cache, k_cache.shape[2])
+    shape = shape_of(k_cache, k_cache.shape[2], 1.0, 1.0)
     _check("pa_copy_blocks", lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_pairs),
                                                 block_pairs.numel() // 2, ctypes.byref(shape), _stream(stream)))
 

@@ -24,11 +24,13 @@ from . import pa
 class DecodeStep:
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_heads: int, num_seqs: int,
                  max_blocks_per_seq: int, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 use_graph: bool = True):
+                 use_graph: bool = True, k_scale: float = 0.0, v_scale: float = 0.0):
         if not (k_cache.is_cuda and v_cache.is_cuda):
             raise ValueError("the KV pool lives on the device")
         self.k_cache, self.v_cache = k_cache, v_cache
-        dev, dt = k_cache.device, k_cache.dtype
+        self.k_scale, self.v_scale = k_scale, v_scale  # for a uint8 (FP8 E4M3) pool
+        dev = k_cache.device
+        dt = torch.bfloat16 if k_cache.dtype == torch.uint8 else k_cache.dtype
         _, _, hk, d = k_cache.shape
         self.num_heads, self.num_seqs = num_heads, num_seqs
         self.max_context_len, self.scale, self.partition_tokens = max_context_len, scale, partition_tokens
@@ -40,7 +42,7 @@ class DecodeStep:
         self.block_tables = torch.empty((num_seqs, max_blocks_per_seq), dtype=torch.int32, device=dev)
         self.context_lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
         nbytes = pa.pa_decode_workspace_bytes(num_seqs, max_context_len, partition_tokens,
-                                              pa.shape_of(k_cache, num_heads))
+                                              pa.shape_of(k_cache, num_heads, k_scale, v_scale))
         self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev) if nbytes else None
         self.stream = torch.cuda.Stream(device=dev)
         self.use_graph = use_graph
@@ -62,9 +64,11 @@ class DecodeStep:
         self.slot_mapping.copy_(slots, non_blocking=True)
         self.block_tables.copy_(tables, non_blocking=True)
         self.context_lens.copy_(lens, non_blocking=True)
-        pa.pa_reshape_and_cache(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping)
+        pa.pa_reshape_and_cache(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping,
+                                k_scale=self.k_scale, v_scale=self.v_scale)
         pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
-                     self.max_context_len, self.scale, self.partition_tokens, self.workspace)
+                     self.max_context_len, self.scale, self.partition_tokens, self.workspace,
+                     k_scale=self.k_scale, v_scale=self.v_scale)
         out.copy_(self.out, non_blocking=True)
 
     def bind(self, q, k_new, v_new, slot_mapping, block_tables, context_lens, out):
