@@ -293,9 +293,10 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
                      int32_t max_blocks_per_seq, const int32_t *cu_q_lens, const int32_t *context_lens,
                      int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens, float scale, const pa_shape *shape,
                      void *stream) {
+    if (shape && shape->kv_fp8) return PA_ERR_UNSUPPORTED;  // FP8 caches are a decode-only layout
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
-    if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128 || shape->kv_fp8) return PA_ERR_UNSUPPORTED;
+    if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (num_seqs < 0 || max_q_len < 0 || num_q_tokens < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
     if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !cu_q_lens || !context_lens)
