@@ -21,8 +21,9 @@
 //    (a [16][D] box of the pool viewed as [NB*16][Hk][D]) into a ring slot,
 //    and an mbarrier counts the bytes. Fetches run NSTAGE blocks ahead, so
 //    the table entry, the HBM fetch and the math of different blocks overlap.
-//  * Lanes own column slices of a row made of CH 16-byte chunks (CH = 2, or 1
-//    for groups of 8 heads to bound registers), interleaved so shared-memory
+//  * Lanes own column slices of a row made of CH chunks of 16 bytes (8 for
+//    FP8 rows with groups of 8 heads; CH = 2, or 1 for groups of 8 heads and
+//    FP8 rows, to bound registers), interleaved so shared-memory
 //    reads are conflict free. L = row_bytes / (16 * CH) lanes cover a row and RS = 32 / L rows are processed per step. q.k
 //    partial sums are folded across the L lanes with a transpose-reduce
 //    (each shuffle step halves the values per lane). Softmax runs in fp32
@@ -46,11 +47,14 @@ template <typename T, int D, int G>
 struct DecodeCfg {
     static constexpr int E = sizeof(T);
     static constexpr int R = D * E;                        // bytes of one token row of one KV head
-    static constexpr int CH = (G >= 8 || E == 1) ? 1 : 2;  // 16-byte chunks a lane owns per row
-    static constexpr int L = R / (16 * CH);                // lanes covering one row
+    // Bytes of one chunk: 16, or 8 for FP8 rows with groups of 8 heads, so that
+    // a lane holds 8 dims per row as for bf16 (16 would spill q and O).
+    static constexpr int CB = (E == 1 && G >= 8) ? 8 : 16;
+    static constexpr int CH = (G >= 8 || E == 1) ? 1 : 2;  // chunks a lane owns per row
+    static constexpr int L = R / (CB * CH);                // lanes covering one row
     static constexpr int RS = 32 / L;                      // rows per warp step
     static constexpr int STEPS = kBlockSize / RS;          // steps per block
-    static constexpr int VE = 16 / E;                      // elements per 16-byte chunk
+    static constexpr int VE = CB / E;                      // elements per chunk
     static constexpr int EPL = CH * VE;                    // elements per lane per row
     static constexpr int STAGE_BYTES = 2 * kBlockSize * R; // K and V of one block
     // Two stages per warp and three CTAs per SM (12 warps) measured faster on
@@ -70,7 +74,7 @@ struct DecodeCfg {
     static constexpr int OFF_S = OFF_BAR + kDecodeWarps * NSTAGE * 8;
     static constexpr int OFF_ML = OFF_S + kDecodeWarps * kBlockSize * G * 4;
     static constexpr int SMEM = OFF_ML + 2 * kDecodeWarps * G * 4;
-    static_assert(R % (16 * CH) == 0 && L >= 1 && L <= 32 && 32 % L == 0, "row must split into lane slices");
+    static_assert(R % (CB * CH) == 0 && L >= 1 && L <= 32 && 32 % L == 0, "row must split into lane slices");
     static_assert(kBlockSize % RS == 0, "rows per step must divide the block");
     static_assert(32 % G == 0 && G <= 8, "group size");
 };
@@ -103,6 +107,21 @@ struct TransposeReduce {
         }
     }
 };
+
+// Widen one CB-byte chunk of a cache row from shared memory to VE / 2 pairs.
+template <typename T, int CB>
+__device__ __forceinline__ void load_chunk(const unsigned char *p, f32x2 *f) {
+    if constexpr (CB == 16) {
+        Widen<T>::apply2(*reinterpret_cast<const uint4 *>(p), f);
+    } else {
+        static_assert(CB == 8 && sizeof(T) == 1, "8-byte chunks are for FP8 rows");
+        const uint2 r = *reinterpret_cast<const uint2 *>(p);
+        f[0] = e4m3x2_to_f32x2(r.x & 0xffffu);
+        f[1] = e4m3x2_to_f32x2(r.x >> 16);
+        f[2] = e4m3x2_to_f32x2(r.y & 0xffffu);
+        f[3] = e4m3x2_to_f32x2(r.y >> 16);
+    }
+}
 
 struct DecodeParams {
     void *out;
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
 
     // Queries of the group, pre-scaled by scale * log2(e), as packed pairs.
     constexpr int P2 = C::EPL / 2;  // packed pairs per lane per row
-    constexpr int VP = C::VE / 2;   // packed pairs per 16-byte chunk
+    constexpr int VP = C::VE / 2;   // packed pairs per chunk
     f32x2 q2[G][P2];
     {
         // the lane's dims in q: the same VE-element chunks as in the cache row
@@ -252,10 +271,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             const int row = st * C::RS + rg;
             f32x2 k2[P2];
 #pragma unroll
-            for (int ch = 0; ch < C::CH; ++ch) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(kb + row * C::R + (ch * C::L + j) * 16);
-                Widen<Tc>::apply2(raw, &k2[ch * VP]);
-            }
+            for (int ch = 0; ch < C::CH; ++ch) load_chunk<Tc, C::CB>(kb + row * C::R + (ch * C::L + j) * C::CB, &k2[ch * VP]);
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 f32x2 s2 = 0ull;
@@ -334,10 +350,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             for (int g = 0; g < G; ++g) pr[g] = s_buf[t * G + g];
             f32x2 v2[P2];
 #pragma unroll
-            for (int ch = 0; ch < C::CH; ++ch) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(vb + t * C::R + (ch * C::L + j) * 16);
-                Widen<Tc>::apply2(raw, &v2[ch * VP]);
-            }
+            for (int ch = 0; ch < C::CH; ++ch) load_chunk<Tc, C::CB>(vb + t * C::R + (ch * C::L + j) * C::CB, &v2[ch * VP]);
             if (t < n_valid) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {

@@ -305,8 +305,9 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_tables, 4) ||
         !aligned(cu_q_lens, 4) || !aligned(context_lens, 4))
         return PA_ERR_ALIGNMENT;
-    return pa::launch_prefill(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, cu_q_lens, context_lens,
-                              num_seqs, max_q_len, num_q_tokens, scale, shape, static_cast<cudaStream_t>(stream));
+    rc = pa::launch_prefill(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, cu_q_lens, context_lens,
+                            num_seqs, max_q_len, num_q_tokens, scale, shape, static_cast<cudaStream_t>(stream));
+    return rc == PA_ERR_CUDA ? cuda_fail(cudaGetLastError()) : rc;  // keep the CUDA error for pa_last_cuda_error
 }
 
 }  // extern "C"

@@ -9,34 +9,38 @@
 // with K/V rows found through the block table, as in decode.
 //
 // How it runs (bf16 in, fp32 accumulate, head_dim 128), warp-specialized:
-//  * A CTA owns two Q tiles of 128 rows. Each row is one of (128 / G) chunk
-//    tokens x the G query heads of one KV head (GQA packing), so every K/V tile
-//    loaded serves all G heads of both Q tiles.
-//  * Warp 0 (producer) streams Q and then 64-key K/V tiles by TMA with 128-byte
-//    swizzle into a 3-stage ring. A tile is four 16-token blocks, and each block
-//    of each 64-column half is one TMA box addressed through the block table.
-//    Blocks past the context (and bad table entries) load from an out-of-range
-//    row, which fills zeros. The producer zeroes the last tile's V rows past the
-//    context before the MMA may read them (0 * NaN would poison O).
-//  * Warp 1 issues the MMAs from one thread: S = Q K^T (M=128, N=64) and
-//    O += P V (M=128, N=128), tcgen05.mma kind::f16, with S and O for both Q
-//    tiles in tensor memory. The order is QK(tile 0, j+1), PV(tile 0, j),
-//    QK(tile 1, j+1), PV(tile 1, j), so one Q tile's softmax overlaps the other
-//    tile's MMAs.
-//  * Warps 4..7 and 8..11 run the softmax of Q tiles 0 and 1; thread = row =
-//    TMEM lane. A thread reads its 64 scores in one tcgen05.ld and releases S
-//    at once. It masks keys past its causal limit, takes the row max, and
-//    computes p = 2^(s*scale*log2(e) - m) with one FMA and one ex2. It writes
-//    P as bf16 into shared memory in the swizzled K-major layout the MMA reads,
-//    and sums the fp32 p in packed pairs. The reference max is replaced (and O
-//    rescaled in TMEM) only when a row max grows by more than 2^8.
-//  * P is double-buffered per Q tile. The softmax of tile j waits only for the
-//    PV of tile j-2 (buffer reuse), and for that of tile j-1 only when it
-//    rescales O.
+//  * A CTA owns up to two Q tiles of 128 rows. Each row is one of (128 / G)
+//    chunk tokens x the G query heads of one KV head (GQA packing), so every
+//    K/V tile loaded serves all G heads of both Q tiles. A chunk too short to
+//    reach the second tile (a decode token, a short verify chunk) runs one.
+//  * Warp 0 (producer) streams Q and then 128-key K/V tiles by TMA with
+//    128-byte swizzle into a 2-stage ring. A tile is eight 16-token blocks, and
+//    each block of each 64-column half is one TMA box addressed through the
+//    block table. Blocks past the context (and bad table entries) load from an
+//    out-of-range row, which fills zeros. The producer zeroes the last tile's V
+//    rows past the context before the MMA may read them (0 * NaN would poison O).
+//  * Warp 1 issues the MMAs from one thread: S = Q K^T (M=128, N=128) and
+//    O += P V (M=128, N=128, K=128), tcgen05.mma kind::f16, with S, P and O of
+//    both Q tiles in tensor memory (512 columns). P is written as bf16 over the
+//    first half of its own S and is the A operand of P V straight from tensor
+//    memory. 128-key tiles keep the QK MMA at full rate (at N=64 it is bound by
+//    shared-memory operand reads) and halve the hand-offs per key.
+//  * The order per tile is PV(tile 0, j), QK(tile 0, j+1), PV(tile 1, j),
+//    QK(tile 1, j+1): one Q tile's softmax overlaps the other tile's MMAs. A QK
+//    overwrites P, so it waits for the P V before it (odone).
+//  * Warps 2..5 and 6..9 run the softmax of Q tiles 0 and 1; thread = row =
+//    TMEM lane; a warp whose rows hold no chunk token only keeps the barrier
+//    protocol. A thread reads its scores in two 64-key halves, masks keys past
+//    its causal limit and computes p = 2^(s*scale*log2(e) - m) with one FMA
+//    and one ex2, summing the fp32 p in packed pairs. The reference max m is
+//    replaced (and O rescaled in TMEM) only when a row max grows by more than
+//    2^8, so the first half is exponentiated before the second is read, and
+//    only re-scaled in the rare case that the second half moves m.
 //  * Hand-offs are mbarriers only: full/empty per ring stage (empties committed
-//    by tcgen05.commit), sfull/sfree for S, pready, and odone per P buffer.
-//    Every wait is bounded and also gives up when another role has aborted. The
-//    MMA thread drains its work before tensor memory is freed.
+//    by tcgen05.commit), and per Q tile sfull (S ready; it also implies the
+//    previous P V is done, so O may be rescaled), pready and odone. Every wait
+//    is bounded and also gives up when another role has aborted. The MMA thread
+//    drains its work before tensor memory is freed.
 #pragma once
 
 #include <math_constants.h>
@@ -70,6 +74,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: the A operand (M rows = TMEM lanes, K
+// along columns, two bf16 per 32-bit column) is read from tensor memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -158,33 +174,38 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 
 // ---- geometry -------------------------------------------------------------------
 
-constexpr int kPfWarps = 12;
+constexpr int kPfWarps = 10;                 // producer, MMA, two groups of 4 softmax warps
 constexpr int kPfThreads = 32 * kPfWarps;
+constexpr int kPfSoftmax0 = 2;               // first softmax warp
 constexpr int kPfM = 128;                    // rows per Q tile (tokens x group heads)
 constexpr int kPfNQ = 2;                     // Q tiles per CTA, ping-ponged
-constexpr int kPfN = 64;                     // keys per K/V tile
+constexpr int kPfN = 128;                    // keys per K/V tile
 constexpr int kPfD = 128;                    // head_dim
-constexpr int kPfNS = 3;                     // K/V pipeline stages
+constexpr int kPfNS = 2;                     // K/V pipeline stages
 constexpr int kPfQHalf = kPfM * 64 * 2;      // a 64-column half of a Q tile: 16 KB
 constexpr int kPfQTile = 2 * kPfQHalf;       // 32 KB
-constexpr int kPfKVHalf = kPfN * 64 * 2;     // a 64-dim half of a K/V tile: 8 KB
-constexpr int kPfKVTile = 2 * kPfKVHalf;     // 16 KB
-constexpr int kPfPTile = kPfM * kPfN * 2;    // P: 128 rows x 64 keys bf16 = 16 KB
+constexpr int kPfKVHalf = kPfN * 64 * 2;     // a 64-dim half of a K/V tile: 16 KB
+constexpr int kPfKVTile = 2 * kPfKVHalf;     // 32 KB
 constexpr int kPfOffQ = 0;
 constexpr int kPfOffK = kPfOffQ + kPfNQ * kPfQTile;
 constexpr int kPfOffV = kPfOffK + kPfNS * kPfKVTile;
-constexpr int kPfOffP = kPfOffV + kPfNS * kPfKVTile;
-constexpr int kPfOffBar = kPfOffP + 2 * kPfNQ * kPfPTile;  // P double-buffered per Q tile
-// mbarriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], vzero, drain, then per Q tile:
-// sfull, sfree, pready, odone[2] (one per P buffer)
+constexpr int kPfOffBar = kPfOffV + kPfNS * kPfKVTile;
+// mbarriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], vzero, drain, then per
+// Q tile: sfull (S ready), pready (P written), odone (the P V of the tile done)
 constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNS, kPfBarVF = kPfBarKE + kPfNS,
               kPfBarVE = kPfBarVF + kPfNS, kPfBarVZ = kPfBarVE + kPfNS, kPfBarDrain = kPfBarVZ + 1,
-              kPfBarTile = kPfBarDrain + 1, kPfTileBars = 5, kPfBars = kPfBarTile + kPfTileBars * kPfNQ;
+              kPfBarTile = kPfBarDrain + 1, kPfTileBars = 3, kPfBars = kPfBarTile + kPfTileBars * kPfNQ;
 constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;  // TMEM base address, abort flag
 constexpr int kPfSmem = kPfOffSlot + 16 + 1024;      // + room to align the base to 1024 B
-constexpr uint32_t kPfTmemCols = 512;                // S_A, S_B (64 each), O_A, O_B (128 each)
-constexpr int kPfBlocksPerTile = kPfN / kBlockSize;  // 4
+// Tensor memory columns: S_A, S_B (128 fp32 each), then O_A, O_B (128 each). P of
+// a Q tile (128 bf16 = 64 columns) overwrites the first half of its own S.
+constexpr uint32_t kPfColP = 0;
+constexpr uint32_t kPfColO = kPfNQ * kPfN;
+constexpr uint32_t kPfTmemCols = 512;
+constexpr int kPfBlocksPerTile = kPfN / kBlockSize;  // 8
+static_assert(kPfColO + kPfNQ * kPfD <= kPfTmemCols, "tensor memory over 512 columns");
 static_assert(kPfSmem <= 232448, "prefill shared memory over the 227 KB limit");
+static_assert(kPfBlocksPerTile <= 32, "one producer lane per block of a tile");
 
 struct PrefillParams {
     void *out;
@@ -198,6 +219,27 @@ struct PrefillParams {
     int num_q_tokens;
     float scale_log2;
 };
+
+// p = 2^(x * sc + nm) for 64 scores of one row: the fp32 p are summed into acc
+// in packed pairs, and the bf16 pairs (keys 2w, 2w+1 in column w) are stored to
+// 32 TMEM columns at taddr.
+__device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, float nm, f32x2 (&acc)[4],
+                                            uint32_t taddr) {
+    float pv[32];
+#pragma unroll
+    for (int w = 0; w < 32; ++w) {
+        const float a0 = fmaf(x[2 * w], sc, nm), a1 = fmaf(x[2 * w + 1], sc, nm);
+        const float p0 = ex2_approx(a0);
+        const float p1 = ex2_approx(a1);
+        add2(acc[w & 3], pack2(p0, p1));
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        pv[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
+    }
+    // finish the sums here: otherwise the compiler keeps the 64 p values alive
+    // into the next half and runs out of registers
+    asm volatile("" : "+l"(acc[0]), "+l"(acc[1]), "+l"(acc[2]), "+l"(acc[3]));
+    tmem_st32(taddr, pv);
+}
 
 // Bounded mbarrier wait that also gives up when another role of the CTA has aborted.
 __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
@@ -243,8 +285,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int ct = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // longest CTAs first
     if (ct >= n_ct) return;
     const int t0 = ct * kPfNQ * TOK;
+    const int n_q = q_len - t0 > TOK ? 2 : 1;  // Q tiles holding chunk tokens (a short chunk uses one)
     const int o = c - q_len;
-    const int kv_end = o + min(t0 + kPfNQ * TOK, q_len);  // keys needed: [0, kv_end)
+    const int kv_end = o + min(t0 + n_q * TOK, q_len);  // keys needed: [0, kv_end)
     const int n_tiles = (kv_end + kPfN - 1) / kPfN;
     const int nblk_seq = (c + kBlockSize - 1) / kBlockSize;
     const bool zero_tail = n_tiles * kPfN > c;  // the last tile holds keys past the context
@@ -271,10 +314,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_init(bar(kPfBarDrain), 1);
         for (int qi = 0; qi < kPfNQ; ++qi) {
             mbar_init(bar(kPfBarTile + kPfTileBars * qi + 0), 1);    // sfull: MMA commit
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // sfree: every softmax thread
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 2), 128);  // pready: every softmax thread
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 3), 1);    // odone, P buffer 0: MMA commit
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 4), 1);    // odone, P buffer 1: MMA commit
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // pready: every softmax thread
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 2), 1);    // odone: MMA commit
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -310,8 +351,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
         };
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar(kPfBarQ), kPfNQ * kPfQTile);
-            for (int qi = 0; qi < kPfNQ; ++qi) {
+            mbar_arrive_expect_tx(bar(kPfBarQ), n_q * kPfQTile);
+            for (int qi = 0; qi < n_q; ++qi) {
                 const uint32_t dq = base_s + kPfOffQ + qi * kPfQTile;
                 const int qrow = q0 + t0 + qi * TOK;
                 tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(kPfBarQ));
@@ -366,7 +407,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
             constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
-            auto issue_qk = [&](int qi, int j) {
+            auto b_tile = [&](int qi, int k) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + k); };
+            auto issue_qk = [&](int qi, int j) {  // S_qi = Q_qi K_j^T
                 const uint32_t qb = base_s + kPfOffQ + qi * kPfQTile;
                 const uint32_t kb = base_s + kPfOffK + (j % kPfNS) * kPfKVTile;
 #pragma unroll
@@ -374,48 +416,46 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     umma_bf16(tmem + qi * kPfN, smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
                               smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
                 }
-                umma_commit(bar(kPfBarTile + kPfTileBars * qi + 0));
+                umma_commit(b_tile(qi, 0));
             };
-            auto issue_pv = [&](int qi, int j) {
-                const uint32_t pb = base_s + kPfOffP + (2 * qi + (j & 1)) * kPfPTile;
+            auto issue_pv = [&](int qi, int j) {  // O_qi += P_qi V_j, P read from tensor memory
+                const uint32_t pt = tmem + qi * kPfN + kPfColP;
                 const uint32_t vb = base_s + kPfOffV + (j % kPfNS) * kPfKVTile;
 #pragma unroll
-                for (int kk = 0; kk < kPfN / 16; ++kk) {
-                    umma_bf16(tmem + 2 * kPfN + qi * kPfD, smem_desc_sw128(pb + kk * 32, 16, 1024),
-                              smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kPfN / 16; ++kk) {  // 16 keys = 8 columns of P
+                    umma_bf16_ts(tmem + kPfColO + qi * kPfD, pt + kk * 8,
+                                 smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(bar(kPfBarTile + kPfTileBars * qi + 3 + (j & 1)));
+                umma_commit(b_tile(qi, 2));
             };
             bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag) && pf_wait(bar(kPfBarKF), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_qk(0, 0);
-                issue_qk(1, 0);
+                for (int qi = 0; qi < n_q; ++qi) issue_qk(qi, 0);
                 umma_commit(bar(kPfBarKE));
             }
             for (int j = 0; j < n_tiles && ok; ++j) {
                 const int s = j % kPfNS, u = j / kPfNS;
                 const int s1 = (j + 1) % kPfNS, u1 = (j + 1) / kPfNS;
                 const bool more = j + 1 < n_tiles;
-                for (int qi = 0; qi < kPfNQ && ok; ++qi) {
-                    // S of the next tile once softmax qi has read this tile's S
-                    if (more) {
-                        ok = pf_wait(bar(kPfBarKF + s1), u1 & 1, abort_flag) &&
-                             pf_wait(bar(kPfBarTile + kPfTileBars * qi + 1), j & 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_qk(qi, j + 1);
-                        if (qi == kPfNQ - 1) umma_commit(bar(kPfBarKE + s1));
-                    }
+                for (int qi = 0; qi < n_q && ok; ++qi) {
                     // O += P V once softmax qi has written P (and rescaled O)
-                    ok = pf_wait(bar(kPfBarTile + kPfTileBars * qi + 2), j & 1, abort_flag);
+                    ok = pf_wait(b_tile(qi, 1), j & 1, abort_flag);
                     if (ok && qi == 0)
                         ok = (j == n_tiles - 1 && zero_tail) ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
                                                              : pf_wait(bar(kPfBarVF + s), u & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(qi, j);
-                    if (qi == kPfNQ - 1) umma_commit(bar(kPfBarVE + s));
+                    if (qi == n_q - 1) umma_commit(bar(kPfBarVE + s));
+                    if (!more) continue;
+                    // the next S overwrites P: wait for this P V to finish reading it
+                    ok = pf_wait(b_tile(qi, 2), j & 1, abort_flag);
+                    if (ok && qi == 0) ok = pf_wait(bar(kPfBarKF + s1), u1 & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(qi, j + 1);
+                    if (qi == n_q - 1) umma_commit(bar(kPfBarKE + s1));
                 }
             }
             // every MMA issued so far completes before tensor memory can be freed
@@ -423,125 +463,142 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_wait(bar(kPfBarDrain), 0);
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ================= softmax: warps 4..7 own Q tile 0, warps 8..11 Q tile 1 =================
-        const int qi = (warp - 4) / 4;
-        const int r = (warp & 3) * 32 + lane;  // row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + qi * kPfN, tO = tmem + 2 * kPfN + qi * kPfD;
+    } else {
+        // ====== softmax: warps 2..5 own Q tile 0, warps 6..9 Q tile 1; thread = row = TMEM lane ======
+        const int qi = (warp - kPfSoftmax0) / 4;
+        const int quad = warp & 3;  // a warp reaches TMEM lanes 32 * (warp % 4) .. + 31
+        const int r = quad * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t tS = tmem + qi * kPfN + lane_base, tO = tmem + kPfColO + qi * kPfD + lane_base;
         const uint32_t b_sfull = bar(kPfBarTile + kPfTileBars * qi + 0);
-        const uint32_t b_sfree = bar(kPfBarTile + kPfTileBars * qi + 1);
-        const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 2);
-        // odone[x] completes when the PV that read P buffer x is done (every other tile)
-        auto b_odone = [&](int x) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + 3 + x); };
-        const int tq = t0 + qi * TOK;                 // first chunk token of this Q tile
+        const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 1);
+        const uint32_t b_odone = bar(kPfBarTile + kPfTileBars * qi + 2);
+        const int tq = t0 + qi * TOK;  // first chunk token of this Q tile
         const int rows_valid = max(0, min(TOK, q_len - tq));
+        // warps whose 32 rows hold no chunk token only keep the barrier protocol
+        const bool active = (quad * 32) / G < rows_valid;
         const int tok = min(tq + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
         const int pos = o + tok;                      // causal limit: keys 0..pos
-        unsigned char *prow0 = base + kPfOffP + 2 * qi * kPfPTile + r * 128;
         float m_ref = -CUDART_INF_F, l_sum = 0.f;
-        bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
+        bool ok = qi < n_q;
+        for (int j = 0; j < n_tiles && ok; ++j) {
             ok = __all_sync(0xffffffffu, pf_wait(b_sfull, j & 1, abort_flag));
             if (!ok) break;
-            tc_fence_after();
-            float s[kPfN];  // raw q.k; scale (> 0) is applied inside the exponent
-            tmem_ld64(tS + lane_base, s);
-            tc_fence_before();
-            mbar_arrive(b_sfree);  // S may be overwritten by the next QK
-            const int key0 = j * kPfN;
-            if (key0 + kPfN - 1 > pos) {
-#pragma unroll
-                for (int i = 0; i < kPfN; ++i)
-                    if (key0 + i > pos) s[i] = -CUDART_INF_F;
-            }
-            float m8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-            for (int i = 8; i < kPfN; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * prm.scale_log2;
-            float alpha = 1.f;
-            if (mx > m_ref + 8.f) {  // lazy: keep the older max unless a score exceeds it by 2^8
-                alpha = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
-                m_ref = mx;
-            }
-            // a rescale needs O stable: the PV of tile j-1 (P buffer (j-1)&1) done
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
-                ok = __all_sync(0xffffffffu, pf_wait(b_odone((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag));
-                if (!ok) break;
+            if (active) {
                 tc_fence_after();
-                {
+                // Scores in two 64-key halves a (keys 0..63) and b (64..127), raw q.k; the
+                // scale (> 0) is applied inside the exponent. Half a is exponentiated
+                // against the reference max as it stands after a, and its P goes over
+                // S columns 0..31 (already read). If half b then raises that max (rare
+                // once a row has warmed up), P of a and its sum are scaled down to the
+                // new max. P of b goes over columns 32..63.
+                const int key0 = j * kPfN;
+                const bool edge = key0 + kPfN - 1 > pos;
+                const float sl2 = prm.scale_log2;
+                float h[64];
+                auto load_half = [&](int half) {  // scores of keys key0 + 64*half .. + 63, masked
+                    tmem_ld64(tS + 64 * half, h);
+                    if (edge) {
 #pragma unroll
+                        for (int i = 0; i < 64; ++i)
+                            if (key0 + 64 * half + i > pos) h[i] = -CUDART_INF_F;
+                    }
+                };
+                auto half_max = [&]() -> float {
+                    float m8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) m8[i] = h[i];
+#pragma unroll
+                    for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], h[i]);
+                    return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+                };
+                auto raise = [&](float mx) -> float {  // lazy: move the max only past a 2^8 margin
+                    if (!(mx > m_ref + 8.f)) return 1.f;
+                    const float f = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
+                    m_ref = mx;
+                    return f;
+                };
+                auto exp_half = [&](f32x2 (&sum)[4], uint32_t col) {
+                    const float nm = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+                    const float sc = m_ref == -CUDART_INF_F ? 0.f : sl2;
+                    pf_exp_half(h, sc, nm, sum, tS + col);
+                };
+                f32x2 acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc[4] = {0ull, 0ull, 0ull, 0ull};
+                load_half(0);
+                float alpha = raise(half_max());  // factor for O and l of the earlier tiles
+                exp_half(acc_a, 0);
+                load_half(1);
+                const float beta = raise(half_max());  // factor for half a of this tile
+                if (__any_sync(0xffffffffu, beta != 1.f)) {
+                    float pa[32];
+                    tmem_ld32(tS, pa);
+#pragma unroll
+                    for (int w = 0; w < 32; ++w) {
+                        const uint32_t u = __float_as_uint(pa[w]);
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(u << 16) * beta,
+                                                                        __uint_as_float(u & 0xffff0000u) * beta);
+                        pa[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
+                    }
+                    tmem_st32(tS, pa);
+                    const f32x2 b2 = pack2(beta, beta);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) mul2(acc_a[e], b2);
+                    alpha *= beta;
+                }
+                exp_half(acc, 32);
+                // O of the earlier tiles takes the same factor as l. S of this tile is
+                // complete, and so is every earlier MMA (the P V of tile j-1
+                // included), so O is stable here.
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
+#pragma unroll 1
                     for (int ch = 0; ch < kPfD / 32; ++ch) {
                         float v[32];
-                        tmem_ld32(tO + lane_base + ch * 32, v);
+                        tmem_ld32(tO + ch * 32, v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(tO + lane_base + ch * 32, v);
+                        tmem_st32(tO + ch * 32, v);
                     }
                 }
-            }
-            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score; the row sum
-            // accumulates the fp32 p in packed pairs
-            // P buffer j&1 is free once the PV of tile j-2 is done
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu, pf_wait(b_odone(j & 1), ((j >> 1) - 1) & 1, abort_flag));
-                if (!ok) break;
-            }
-            unsigned char *prow = prow0 + (j & 1) * kPfPTile;
-            const float nm = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-            const float sc = m_ref == -CUDART_INF_F ? 0.f : prm.scale_log2;
-            f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int cc = 0; cc < kPfN / 8; ++cc) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2_approx(fmaf(s[cc * 8 + 2 * e], sc, nm));
-                    const float p1 = ex2_approx(fmaf(s[cc * 8 + 2 * e + 1], sc, nm));
-                    add2(acc[e], pack2(p0, p1));
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                }
-                *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                for (int e = 0; e < 4; ++e) add2(acc[e], acc_a[e]);
+                add2(acc[0], acc[1]);
+                add2(acc[2], acc[3]);
+                add2(acc[0], acc[2]);
+                float lo, hi;
+                unpack2(acc[0], lo, hi);
+                l_sum = l_sum * alpha + (lo + hi);
+                tc_fence_before();  // P and O visible to the MMA issued after the barrier
             }
-            add2(acc[0], acc[1]);
-            add2(acc[2], acc[3]);
-            add2(acc[0], acc[2]);
-            float lo, hi;
-            unpack2(acc[0], lo, hi);
-            l_sum = l_sum * alpha + (lo + hi);
-            fence_async_smem();  // P visible to the tensor core
-            tc_fence_before();
             mbar_arrive(b_pready);
         }
         // ---- epilogue: out = O / l for the valid rows ----
-        if (ok) ok = __all_sync(0xffffffffu, pf_wait(b_odone((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, abort_flag));
-        if (ok) {
-            tc_fence_after();
-            const bool row_ok = r / G < rows_valid;
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            const int orow = row_ok ? q0 + tq + r / G : q0;
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
-                                 (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
+        if (ok && active) {
+            ok = __all_sync(0xffffffffu, pf_wait(b_odone, (n_tiles - 1) & 1, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                const bool row_ok = r / G < rows_valid;
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const int orow = row_ok ? q0 + tq + r / G : q0;
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
+                                     (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
+#pragma unroll 1
+                for (int ch = 0; ch < kPfD / 32; ++ch) {  // 32 columns at a time bounds registers
+                    float v[32];
+                    tmem_ld32(tO + ch * 32, v);
 #pragma unroll
-            for (int ch = 0; ch < kPfD / 32; ++ch) {
-                float v[32];
-                tmem_ld32(tO + lane_base + ch * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    uint4 pkt;
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i] * inv, v[i + 1] * inv);
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[i + 2] * inv, v[i + 3] * inv);
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[i + 4] * inv, v[i + 5] * inv);
-                    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[i + 6] * inv, v[i + 7] * inv);
-                    pkt.x = *reinterpret_cast<uint32_t *>(&h0);
-                    pkt.y = *reinterpret_cast<uint32_t *>(&h1);
-                    pkt.z = *reinterpret_cast<uint32_t *>(&h2);
-                    pkt.w = *reinterpret_cast<uint32_t *>(&h3);
-                    if (row_ok) *reinterpret_cast<uint4 *>(dst + ch * 32 + i) = pkt;
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 pkt;
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i] * inv, v[i + 1] * inv);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[i + 2] * inv, v[i + 3] * inv);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[i + 4] * inv, v[i + 5] * inv);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[i + 6] * inv, v[i + 7] * inv);
+                        pkt.x = *reinterpret_cast<uint32_t *>(&h0);
+                        pkt.y = *reinterpret_cast<uint32_t *>(&h1);
+                        pkt.z = *reinterpret_cast<uint32_t *>(&h2);
+                        pkt.w = *reinterpret_cast<uint32_t *>(&h3);
+                        if (row_ok) *reinterpret_cast<uint4 *>(dst + ch * 32 + i) = pkt;
+                    }
                 }
             }
         }
