@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
 WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny",
-             "copy_blocks", "swap_blocks", "decode_batch_fp8"]
+             "copy_blocks", "swap_blocks", "decode_batch_fp8", "varlen_step", "spec_verify"]
 FP8_K_SCALE, FP8_V_SCALE = 0.02, 1.0 / 48.0
 BLOCK_WORKLOADS = ("copy_blocks", "swap_blocks")
 BLOCK_PAIRS = 2048
@@ -314,9 +314,16 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 
+# Workloads whose whole attention is one pa_prefill_chunk launch over every
+# sequence (decode tokens as chunks of 1, verify chunks, prefill chunks).
+ONE_LAUNCH = ("varlen_step", "spec_verify")
+
+
 def make_workload(name):
     if name == "decode_batch_fp8":
         return W.decode_batch()
+    if name == "varlen_step":  # the mixed step's sequences, attended in one launch
+        return W.mixed_step()
     if name not in W.CONFIGS:
         raise SystemExit("unknown workload %s (one of %s)" % (name, ", ".join(WORKLOADS)))
     return W.CONFIGS[name]()
@@ -396,12 +403,23 @@ def run_ours(args):
         pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
                             case.scale)
 
+    one = args.workload in ONE_LAUNCH
+    out_all = torch.empty_like(q)
+    max_q_all = int(case.q_lens.max())
+
+    def do_all():  # every sequence's chunk, decode tokens included, in one launch
+        pa.pa_prefill_chunk(out_all, q, k_cache, v_cache, tables, cu, lens, max_q_all, case.scale)
+
     parts = [("write", do_write)]
-    if len(pre):
-        parts.append(("prefill", do_prefill))
-    if len(dec):
-        parts.append(("decode", do_decode))
-    launches_per_step = 1 + (1 if len(pre) else 0) + (decode_kernels if len(dec) else 0)
+    if one:
+        parts.append(("attention", do_all))
+        launches_per_step = 2
+    else:
+        if len(pre):
+            parts.append(("prefill", do_prefill))
+        if len(dec):
+            parts.append(("decode", do_decode))
+        launches_per_step = 1 + (1 if len(pre) else 0) + (decode_kernels if len(dec) else 0)
 
     # one graph for the whole step (the headline), one per part (breakdown, roofline)
     graphs = []
@@ -539,7 +557,7 @@ def run_ours(args):
     clocks = sampler.summary(wall0, wall1) if sampler else None
     peak, peak_kind = load_peak()
     roof = None
-    if len(dec):
+    if not one and len(dec):
         t_dec = per_part["decode"] / args.steps
         achieved = nbytes["decode"] / t_dec / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
@@ -570,7 +588,32 @@ def run_ours(args):
             "ms_per_part": parts_ms, "step_bytes": nbytes, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
             "wall_s_timed_region": wall1 - wall0}
-    if len(pre):
+    if one:
+        # One launch does the decode tokens (HBM-bound) and the chunks (tensor-bound
+        # when long). Its floor is the chunks' FLOPs at the bf16 peak plus the decode
+        # tokens' bytes at the copy bandwidth; a launch of verify chunks alone is
+        # HBM-bound (a few rows per KV head).
+        t_one = per_part["attention"] / args.steps
+        tpeak, tkind = load_peak("bf16_tflops")
+        f = prefill_flops(case, pre)
+        attn_bytes = nbytes["decode"] + nbytes["prefill"]
+        long_chunks = [b for b in pre if int(case.q_lens[b]) > 64]
+        f_long = prefill_flops(case, long_chunks)
+        short_bytes = attn_bytes - (step_bytes(case, dec, np.asarray(long_chunks, np.int64))["prefill"]
+                                    if long_chunks else 0)
+        t_floor = f_long / (tpeak * 1e12) + short_bytes / (peak * 1e9)
+        roof = {"bound": "hbm" if not long_chunks else "hbm+tensor",
+                "achieved": attn_bytes / t_one / 1e9 if not long_chunks else t_floor / t_one,
+                "peak": peak if not long_chunks else 1.0,
+                "unit": "GB/s" if not long_chunks else "fraction of the summed floor",
+                "frac": t_floor / t_one, "traffic": None,
+                "kernel": "prefill_kernel (tcgen05), one launch over every sequence",
+                "algorithmic_bytes_per_launch": attn_bytes, "flops_per_launch": f,
+                "floor_us": t_floor * 1e6, "us_per_launch": t_one * 1e6,
+                "peak_kind": "measured (MEASURED_PEAKS.json hbm_gbs%s)" % (
+                    "" if not long_chunks else " and bf16_tflops")}
+        line["roofline"] = roof
+    if not one and len(pre):
         f = prefill_flops(case, pre)
         t_pre = per_part["prefill"] / args.steps
         tpeak, tkind = load_peak("bf16_tflops")

@@ -13,10 +13,11 @@
 //    chunk tokens x the G query heads of one KV head (GQA packing), so every
 //    K/V tile loaded serves all G heads of both Q tiles. A chunk too short to
 //    reach the second tile (a decode token, a short verify chunk) runs one.
-//  * Warp 0 (producer) streams Q and then 128-key K/V tiles by TMA with
-//    128-byte swizzle into a 2-stage ring. A tile is eight 16-token blocks, and
-//    each block of each 64-column half is one TMA box addressed through the
-//    block table. Blocks past the context (and bad table entries) load from an
+//  * Warp 0 streams Q and then 128-key K tiles by TMA with 128-byte swizzle
+//    into a 2-stage ring, and warp 10 the V tiles into a 3-stage ring, so
+//    neither load waits behind the other's free stage. A tile is eight 16-token
+//    blocks, and each block of each 64-column half is one TMA box addressed
+//    through the block table. Blocks past the context (and bad table entries) load from an
 //    out-of-range row, which fills zeros. The producer zeroes the last tile's V
 //    rows past the context before the MMA may read them (0 * NaN would poison O).
 //  * Warp 1 issues the MMAs from one thread: S = Q K^T (M=128, N=128) and
@@ -28,6 +29,12 @@
 //  * The order per tile is PV(tile 0, j), QK(tile 0, j+1), PV(tile 1, j),
 //    QK(tile 1, j+1): one Q tile's softmax overlaps the other tile's MMAs. A QK
 //    overwrites P, so it waits for the P V before it (odone).
+//  * A CTA with one Q tile and two or more K/V tiles splits: slot 1 (the second
+//    S/O pair in TMEM and its softmax warps) runs the same queries over the odd
+//    K/V tiles, slot 0 over the even ones, and the two (m, l, O) merge in the
+//    epilogue (slot 1 hands m and l over in shared memory; slot 0 reads its O
+//    from TMEM). Decode tokens and short verify chunks in a varlen batch then
+//    keep two chains in flight per CTA without a second kernel.
 //  * Warps 2..5 and 6..9 run the softmax of Q tiles 0 and 1; thread = row =
 //    TMEM lane; a warp whose rows hold no chunk token only keeps the barrier
 //    protocol. A thread reads its scores in two 64-key halves, masks keys past
@@ -174,29 +181,32 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 
 // ---- geometry -------------------------------------------------------------------
 
-constexpr int kPfWarps = 10;                 // producer, MMA, two groups of 4 softmax warps
+constexpr int kPfWarps = 11;                 // K producer, MMA, 2 x 4 softmax warps, V producer
 constexpr int kPfThreads = 32 * kPfWarps;
 constexpr int kPfSoftmax0 = 2;               // first softmax warp
+constexpr int kPfVWarp = 10;                 // the V producer
 constexpr int kPfM = 128;                    // rows per Q tile (tokens x group heads)
 constexpr int kPfNQ = 2;                     // Q tiles per CTA, ping-ponged
 constexpr int kPfN = 128;                    // keys per K/V tile
 constexpr int kPfD = 128;                    // head_dim
-constexpr int kPfNS = 2;                     // K/V pipeline stages
+constexpr int kPfNSK = 2;                    // K pipeline stages
+constexpr int kPfNSV = 3;                    // V pipeline stages (a V tile is held longest)
 constexpr int kPfQHalf = kPfM * 64 * 2;      // a 64-column half of a Q tile: 16 KB
 constexpr int kPfQTile = 2 * kPfQHalf;       // 32 KB
 constexpr int kPfKVHalf = kPfN * 64 * 2;     // a 64-dim half of a K/V tile: 16 KB
 constexpr int kPfKVTile = 2 * kPfKVHalf;     // 32 KB
 constexpr int kPfOffQ = 0;
 constexpr int kPfOffK = kPfOffQ + kPfNQ * kPfQTile;
-constexpr int kPfOffV = kPfOffK + kPfNS * kPfKVTile;
-constexpr int kPfOffBar = kPfOffV + kPfNS * kPfKVTile;
-// mbarriers: q, kfull[NS], kempty[NS], vfull[NS], vempty[NS], vzero, drain, then per
-// Q tile: sfull (S ready), pready (P written), odone (the P V of the tile done)
-constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNS, kPfBarVF = kPfBarKE + kPfNS,
-              kPfBarVE = kPfBarVF + kPfNS, kPfBarVZ = kPfBarVE + kPfNS, kPfBarDrain = kPfBarVZ + 1,
+constexpr int kPfOffV = kPfOffK + kPfNSK * kPfKVTile;
+constexpr int kPfOffBar = kPfOffV + kPfNSV * kPfKVTile;
+// mbarriers: q, kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], vzero, drain, then
+// per Q tile: sfull (S ready), pready (P written), odone (the P V of the tile done)
+constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNSK, kPfBarVF = kPfBarKE + kPfNSK,
+              kPfBarVE = kPfBarVF + kPfNSV, kPfBarVZ = kPfBarVE + kPfNSV, kPfBarDrain = kPfBarVZ + 1,
               kPfBarTile = kPfBarDrain + 1, kPfTileBars = 3, kPfBars = kPfBarTile + kPfTileBars * kPfNQ;
 constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;  // TMEM base address, abort flag
-constexpr int kPfSmem = kPfOffSlot + 16 + 1024;      // + room to align the base to 1024 B
+constexpr int kPfOffML = kPfOffSlot + 16;            // (m, l) of slot 1 per row, for the split merge
+constexpr int kPfSmem = kPfOffML + 2 * kPfM * 4 + 1024;  // + room to align the base to 1024 B
 // Tensor memory columns: S_A, S_B (128 fp32 each), then O_A, O_B (128 each). P of
 // a Q tile (128 bf16 = 64 columns) overwrites the first half of its own S.
 constexpr uint32_t kPfColP = 0;
@@ -217,6 +227,7 @@ struct PrefillParams {
     int num_heads;
     int num_kv_heads;
     int num_q_tokens;
+    int num_seqs;
     float scale_log2;
 };
 
@@ -241,6 +252,34 @@ __device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, floa
     tmem_st32(taddr, pv);
 }
 
+// Work slots of a varlen launch: sequence b owns the slots starting at
+// S_b = cu_q_lens[b] / per_cta + b (per_cta = chunk tokens one CTA covers), and
+// uses the first ceil(q_len_b / per_cta) of them. S is strictly increasing and
+// S_{b+1} - S_b >= ceil(q_len_b / per_cta), so num_q_tokens / per_cta + num_seqs
+// slots cover every sequence and at most one slot per sequence stays empty (a
+// grid of max tiles x sequences would leave most decode-token CTAs empty).
+// Returns the largest b with S_b <= w: each step the warp probes 32 evenly spaced
+// candidates and keeps the interval after the last one at or below w.
+__device__ __forceinline__ int pf_find_seq(const int *cu_q_lens, int num_seqs, int per_cta, int w, int lane) {
+    int lo = 0, hi = num_seqs;  // S_lo <= w (S_0 = 0); the answer lies in [lo, hi)
+    while (hi - lo > 1) {
+        const int step = (hi - lo + 31) / 32;
+        const int cand = lo + lane * step;
+        const bool le = cand < hi && __ldg(cu_q_lens + cand) / per_cta + cand <= w;
+        const unsigned m = __ballot_sync(0xffffffffu, le);
+        const int last = m ? 31 - __clz(m) : 0;
+        lo += last * step;
+        hi = min(hi, lo + step);
+    }
+    return lo;
+}
+
+// Compile-time tag for the split and unsplit copies of the kernel's roles.
+template <bool B>
+struct PfSplit {
+    static constexpr bool value = B;
+};
+
 // Bounded mbarrier wait that also gives up when another role of the CTA has aborted.
 __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -261,18 +300,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const PrefillParams prm, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     constexpr int TOK = kPfM / G;  // chunk tokens per Q tile
-    const int b = blockIdx.z, hk = blockIdx.y;
+    constexpr int PER_CTA = kPfNQ * TOK;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    // grid.x = slots x KV heads, KV head fastest, so the slots of one chunk (its
+    // longest tile pairs first) start together
+    const int hk = static_cast<int>(blockIdx.x % static_cast<unsigned>(prm.num_kv_heads));
+    const int w = static_cast<int>(blockIdx.x / static_cast<unsigned>(prm.num_kv_heads));
 
     // Launched as a programmatic dependent: wait for the previous kernel (e.g. the
     // cache write of this chunk) before reading any input.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---- per-sequence geometry (uniform over the CTA) ----
+    // ---- this CTA's sequence and tile pair (every warp finds the same) ----
+    const int b = pf_find_seq(prm.cu_q_lens, prm.num_seqs, PER_CTA, w, lane);
     const int q0 = __ldg(prm.cu_q_lens + b), q1 = __ldg(prm.cu_q_lens + b + 1);
+    const int slot = w - (q0 / PER_CTA + b);  // 0 .. of this sequence's slots
     const int q_len = q1 - q0;
     const int c = __ldg(prm.context_lens + b);
-    const bool first = blockIdx.x == 0 && hk == 0 && tid == 0;
+    const bool first = slot == 0 && hk == 0 && tid == 0;
     if (q_len < 0 || q_len > c || q1 > prm.num_q_tokens) {
         if (first) flag_status(PA_STATUS_BAD_QUERY);
         return;
@@ -281,14 +326,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (first) flag_status(PA_STATUS_BAD_CONTEXT);
         return;
     }
-    const int n_ct = (q_len + kPfNQ * TOK - 1) / (kPfNQ * TOK);
-    const int ct = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // longest CTAs first
-    if (ct >= n_ct) return;
+    const int n_ct = (q_len + PER_CTA - 1) / PER_CTA;
+    if (slot >= n_ct) return;
+    const int ct = n_ct - 1 - slot;  // longest tile pairs first
     const int t0 = ct * kPfNQ * TOK;
     const int n_q = q_len - t0 > TOK ? 2 : 1;  // Q tiles holding chunk tokens (a short chunk uses one)
     const int o = c - q_len;
     const int kv_end = o + min(t0 + n_q * TOK, q_len);  // keys needed: [0, kv_end)
     const int n_tiles = (kv_end + kPfN - 1) / kPfN;
+    // Split: a CTA with one Q tile and two or more K/V tiles runs the second slot
+    // (its TMEM, its softmax warps) on the same queries over the odd K/V tiles,
+    // the first slot takes the even ones, and the two (m, l, O) merge at the end.
+    // Decode tokens and short verify chunks then keep two chains in flight.
+    const bool split_cta = n_q == 1 && n_tiles >= 2;
     const int nblk_seq = (c + kBlockSize - 1) / kBlockSize;
     const bool zero_tail = n_tiles * kPfN > c;  // the last tile holds keys past the context
 
@@ -304,9 +354,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     if (tid == 0) {
         mbar_init(bar(kPfBarQ), 1);
-        for (int i = 0; i < kPfNS; ++i) {
+        for (int i = 0; i < kPfNSK; ++i) {
             mbar_init(bar(kPfBarKF + i), 1);
             mbar_init(bar(kPfBarKE + i), 1);
+        }
+        for (int i = 0; i < kPfNSV; ++i) {
             mbar_init(bar(kPfBarVF + i), 1);
             mbar_init(bar(kPfBarVE + i), 1);
         }
@@ -326,273 +378,322 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ================= producer: TMA loads of Q and K/V tiles =================
-        const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq;
-        const int oob_row = static_cast<int>(prm.num_blocks * kBlockSize);  // past the pool: TMA fills zeros
-        auto tile_row = [&](int t) -> int {  // pool row of block `lane` of tile t
-            if (lane >= kPfBlocksPerTile || t >= n_tiles) return oob_row;
-            const int lb = t * kPfBlocksPerTile + lane;
-            if (lb >= nblk_seq) return oob_row;
-            const int pb = __ldg(trow + lb);
-            if (pb < 0 || pb >= prm.num_blocks) {
-                flag_status(PA_STATUS_BAD_BLOCK_ID);
-                return oob_row;
-            }
-            return pb * kBlockSize;
-        };
-        auto load_kv = [&](const CUtensorMap *tm, uint32_t dst, uint32_t full, int row) {
-            if (lane == 0) mbar_arrive_expect_tx(full, kPfKVTile);
-            __syncwarp();
-            if (lane < kPfBlocksPerTile) {
-                const uint32_t d = dst + lane * (kBlockSize * 128);  // 16 rows of 128 B
-                tma_load_3d(d, tm, 0, hk, row, full);
-                tma_load_3d(d + kPfKVHalf, tm, 64, hk, row, full);
-            }
-        };
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(kPfBarQ), n_q * kPfQTile);
-            for (int qi = 0; qi < n_q; ++qi) {
-                const uint32_t dq = base_s + kPfOffQ + qi * kPfQTile;
-                const int qrow = q0 + t0 + qi * TOK;
-                tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(kPfBarQ));
-                tma_load_3d(dq + kPfQHalf, &tm_q, 64, hk * G, qrow, bar(kPfBarQ));
-            }
-        }
-        int row = tile_row(0);
-        int issued = 0;
-        bool ok = true;
-        for (int j = 0; j < n_tiles && ok; ++j) {
-            const int s = j % kPfNS, u = j / kPfNS;
-            const int row_next = tile_row(j + 1);  // fetched while this tile's loads go out
-            if (u >= 1) ok = pf_wait(bar(kPfBarKE + s), (u - 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            load_kv(&tm_k, base_s + kPfOffK + s * kPfKVTile, bar(kPfBarKF + s), row);
-            if (u >= 1) ok = pf_wait(bar(kPfBarVE + s), (u - 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) {
-                issued = 2 * j + 1;
-                break;
-            }
-            load_kv(&tm_v, base_s + kPfOffV + s * kPfKVTile, bar(kPfBarVF + s), row);
-            issued = 2 * j + 2;
-            if (j == n_tiles - 1 && zero_tail) {
-                // keys past the context: their V rows (tail slots) may hold anything, and
-                // 0 * NaN would poison O, so zero them before the MMA reads the tile
-                ok = __all_sync(0xffffffffu, pf_wait(bar(kPfBarVF + s), u & 1, abort_flag));
-                if (ok) {
-                    const int first_bad = max(0, c - j * kPfN);
-                    unsigned char *vt = base + kPfOffV + s * kPfKVTile;
-                    for (int i = lane; i < (kPfN - first_bad) * 16; i += 32) {
-                        const int r = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
-                        *reinterpret_cast<uint4 *>(vt + half * kPfKVHalf + r * 128 + chunk * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(kPfBarVZ));
+    // The roles are compiled twice, split and unsplit, and each CTA runs one copy:
+    // a runtime flag in the inner loops cost the unsplit prefill about 10 %.
+    auto roles = [&](auto split_tag) {
+        constexpr bool split = decltype(split_tag)::value;
+        const int n_slots = split ? 2 : n_q;
+        if (warp == 0 || warp == kPfVWarp) {
+            // ====== producers: warp 0 loads Q and the K tiles, the V warp the V tiles (TMA) ======
+            // Separate rings let a K tile load as soon as its stage is free, whatever V waits on.
+            const bool is_v = warp == kPfVWarp;
+            const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq;
+            const int oob_row = static_cast<int>(prm.num_blocks * kBlockSize);  // past the pool: TMA fills zeros
+            auto tile_row = [&](int t) -> int {  // pool row of block `lane` of tile t
+                if (lane >= kPfBlocksPerTile || t >= n_tiles) return oob_row;
+                const int lb = t * kPfBlocksPerTile + lane;
+                if (lb >= nblk_seq) return oob_row;
+                const int pb = __ldg(trow + lb);
+                if (pb < 0 || pb >= prm.num_blocks) {
+                    flag_status(PA_STATUS_BAD_BLOCK_ID);
+                    return oob_row;
                 }
-            }
-            row = row_next;
-        }
-        if (*abort_flag) {  // let loads nobody consumed land before the CTA exits
-            for (int i = 0; i < issued; ++i) {
-                const int j = i / 2, s = j % kPfNS, u = j / kPfNS;
-                mbar_wait(bar((i & 1 ? kPfBarVF : kPfBarKF) + s), u & 1);
-            }
-        }
-    } else if (warp == 1) {
-        // ================= MMA issue (one thread) =================
-        if (lane == 0) {
-            constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
-            constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
-            auto b_tile = [&](int qi, int k) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + k); };
-            auto issue_qk = [&](int qi, int j) {  // S_qi = Q_qi K_j^T
-                const uint32_t qb = base_s + kPfOffQ + qi * kPfQTile;
-                const uint32_t kb = base_s + kPfOffK + (j % kPfNS) * kPfKVTile;
-#pragma unroll
-                for (int kk = 0; kk < kPfD / 16; ++kk) {
-                    umma_bf16(tmem + qi * kPfN, smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
-                              smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
-                }
-                umma_commit(b_tile(qi, 0));
+                return pb * kBlockSize;
             };
-            auto issue_pv = [&](int qi, int j) {  // O_qi += P_qi V_j, P read from tensor memory
-                const uint32_t pt = tmem + qi * kPfN + kPfColP;
-                const uint32_t vb = base_s + kPfOffV + (j % kPfNS) * kPfKVTile;
-#pragma unroll
-                for (int kk = 0; kk < kPfN / 16; ++kk) {  // 16 keys = 8 columns of P
-                    umma_bf16_ts(tmem + kPfColO + qi * kPfD, pt + kk * 8,
-                                 smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+            const CUtensorMap *tm = is_v ? &tm_v : &tm_k;
+            const int ns = is_v ? kPfNSV : kPfNSK;
+            const uint32_t ring = base_s + (is_v ? kPfOffV : kPfOffK);
+            const int b_full = is_v ? kPfBarVF : kPfBarKF, b_empty = is_v ? kPfBarVE : kPfBarKE;
+            auto load_tile = [&](int s, int row) {
+                const uint32_t full = bar(b_full + s);
+                if (lane == 0) mbar_arrive_expect_tx(full, kPfKVTile);
+                __syncwarp();
+                if (lane < kPfBlocksPerTile) {
+                    const uint32_t d = ring + s * kPfKVTile + lane * (kBlockSize * 128);  // 16 rows of 128 B
+                    tma_load_3d(d, tm, 0, hk, row, full);
+                    tma_load_3d(d + kPfKVHalf, tm, 64, hk, row, full);
                 }
-                umma_commit(b_tile(qi, 2));
             };
-            bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag) && pf_wait(bar(kPfBarKF), 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                for (int qi = 0; qi < n_q; ++qi) issue_qk(qi, 0);
-                umma_commit(bar(kPfBarKE));
+            if (!is_v && lane == 0) {
+                mbar_arrive_expect_tx(bar(kPfBarQ), n_q * kPfQTile);
+                for (int qi = 0; qi < n_q; ++qi) {
+                    const uint32_t dq = base_s + kPfOffQ + qi * kPfQTile;
+                    const int qrow = q0 + t0 + qi * TOK;
+                    tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(kPfBarQ));
+                    tma_load_3d(dq + kPfQHalf, &tm_q, 64, hk * G, qrow, bar(kPfBarQ));
+                }
             }
+            int row = tile_row(0);
+            int issued = 0;
+            bool ok = true;
             for (int j = 0; j < n_tiles && ok; ++j) {
-                const int s = j % kPfNS, u = j / kPfNS;
-                const int s1 = (j + 1) % kPfNS, u1 = (j + 1) / kPfNS;
-                const bool more = j + 1 < n_tiles;
-                for (int qi = 0; qi < n_q && ok; ++qi) {
-                    // O += P V once softmax qi has written P (and rescaled O)
-                    ok = pf_wait(b_tile(qi, 1), j & 1, abort_flag);
-                    if (ok && qi == 0)
-                        ok = (j == n_tiles - 1 && zero_tail) ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
-                                                             : pf_wait(bar(kPfBarVF + s), u & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(qi, j);
-                    if (qi == n_q - 1) umma_commit(bar(kPfBarVE + s));
-                    if (!more) continue;
-                    // the next S overwrites P: wait for this P V to finish reading it
-                    ok = pf_wait(b_tile(qi, 2), j & 1, abort_flag);
-                    if (ok && qi == 0) ok = pf_wait(bar(kPfBarKF + s1), u1 & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_qk(qi, j + 1);
-                    if (qi == n_q - 1) umma_commit(bar(kPfBarKE + s1));
+                const int s = j % ns, u = j / ns;
+                const int row_next = tile_row(j + 1);  // fetched while this tile's loads go out
+                if (u >= 1) ok = pf_wait(bar(b_empty + s), (u - 1) & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                load_tile(s, row);
+                issued = j + 1;
+                if (is_v && j == n_tiles - 1 && zero_tail) {
+                    // keys past the context: their V rows (tail slots) may hold anything, and
+                    // 0 * NaN would poison O, so zero them before the MMA reads the tile
+                    ok = __all_sync(0xffffffffu, pf_wait(bar(b_full + s), u & 1, abort_flag));
+                    if (ok) {
+                        const int first_bad = max(0, c - j * kPfN);
+                        unsigned char *vt = base + kPfOffV + s * kPfKVTile;
+                        for (int i = lane; i < (kPfN - first_bad) * 16; i += 32) {
+                            const int r = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
+                            *reinterpret_cast<uint4 *>(vt + half * kPfKVHalf + r * 128 + chunk * 16) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(kPfBarVZ));
+                    }
                 }
+                row = row_next;
             }
-            // every MMA issued so far completes before tensor memory can be freed
-            umma_commit(bar(kPfBarDrain));
-            mbar_wait(bar(kPfBarDrain), 0);
-        }
-        __syncwarp();
-    } else {
-        // ====== softmax: warps 2..5 own Q tile 0, warps 6..9 Q tile 1; thread = row = TMEM lane ======
-        const int qi = (warp - kPfSoftmax0) / 4;
-        const int quad = warp & 3;  // a warp reaches TMEM lanes 32 * (warp % 4) .. + 31
-        const int r = quad * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t tS = tmem + qi * kPfN + lane_base, tO = tmem + kPfColO + qi * kPfD + lane_base;
-        const uint32_t b_sfull = bar(kPfBarTile + kPfTileBars * qi + 0);
-        const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 1);
-        const uint32_t b_odone = bar(kPfBarTile + kPfTileBars * qi + 2);
-        const int tq = t0 + qi * TOK;  // first chunk token of this Q tile
-        const int rows_valid = max(0, min(TOK, q_len - tq));
-        // warps whose 32 rows hold no chunk token only keep the barrier protocol
-        const bool active = (quad * 32) / G < rows_valid;
-        const int tok = min(tq + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
-        const int pos = o + tok;                      // causal limit: keys 0..pos
-        float m_ref = -CUDART_INF_F, l_sum = 0.f;
-        bool ok = qi < n_q;
-        for (int j = 0; j < n_tiles && ok; ++j) {
-            ok = __all_sync(0xffffffffu, pf_wait(b_sfull, j & 1, abort_flag));
-            if (!ok) break;
-            if (active) {
+            if (*abort_flag) {  // let loads nobody consumed land before the CTA exits
+                for (int i = 0; i < issued; ++i) mbar_wait(bar(b_full + i % ns), (i / ns) & 1);
+            }
+        } else if (warp == 1) {
+            // ================= MMA issue (one thread) =================
+            if (lane == 0) {
+                constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
+                constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
+                auto b_tile = [&](int qi, int k) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + k); };
+                // slot qi takes K/V tiles tile_of(qi, 0 .. n_of(qi) - 1); `last` marks the
+                // slot after whose MMA a K/V stage may be refilled
+                auto n_of = [&](int qi) -> int { return split ? (n_tiles - qi + 1) / 2 : n_tiles; };
+                auto tile_of = [&](int qi, int i) -> int { return split ? 2 * i + qi : i; };
+                const auto last = [&](int qi) -> bool { return split || qi == n_q - 1; };
+                auto issue_qk = [&](int qi, int j) {  // S_qi = Q K_j^T
+                    const uint32_t qb = base_s + kPfOffQ + (split ? 0 : qi) * kPfQTile;
+                    const uint32_t kb = base_s + kPfOffK + (j % kPfNSK) * kPfKVTile;
+    #pragma unroll
+                    for (int kk = 0; kk < kPfD / 16; ++kk) {
+                        umma_bf16(tmem + qi * kPfN,
+                                  smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
+                                  smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK,
+                                  kk > 0);
+                    }
+                    umma_commit(b_tile(qi, 0));
+                    if (last(qi)) umma_commit(bar(kPfBarKE + j % kPfNSK));
+                };
+                auto issue_pv = [&](int qi, int j, bool acc) {  // O_qi (+)= P_qi V_j, P read from tensor memory
+                    const uint32_t pt = tmem + qi * kPfN + kPfColP;
+                    const uint32_t vb = base_s + kPfOffV + (j % kPfNSV) * kPfKVTile;
+    #pragma unroll
+                    for (int kk = 0; kk < kPfN / 16; ++kk) {  // 16 keys = 8 columns of P
+                        umma_bf16_ts(tmem + kPfColO + qi * kPfD, pt + kk * 8,
+                                     smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV,
+                                     (acc || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(b_tile(qi, 2));
+                    if (last(qi)) umma_commit(bar(kPfBarVE + j % kPfNSV));
+                };
+                // the first slot to read a K/V tile waits for it; in the unsplit order the
+                // second slot's MMA on the same tile comes after the first one's
+                auto wait_k = [&](int qi, int j) {
+                    return (qi > 0 && !split) || pf_wait(bar(kPfBarKF + j % kPfNSK), (j / kPfNSK) & 1, abort_flag);
+                };
+                auto wait_v = [&](int qi, int j) {
+                    if (qi > 0 && !split) return true;
+                    return (j == n_tiles - 1 && zero_tail)
+                               ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
+                               : pf_wait(bar(kPfBarVF + j % kPfNSV), (j / kPfNSV) & 1, abort_flag);
+                };
+                bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag);
+                for (int qi = 0; qi < n_slots && ok; ++qi) {
+                    ok = wait_k(qi, tile_of(qi, 0));
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(qi, tile_of(qi, 0));
+                }
+                const int rounds = n_of(0);
+                for (int i = 0; i < rounds && ok; ++i) {
+                    for (int qi = 0; qi < n_slots && ok; ++qi) {
+                        if (i >= n_of(qi)) continue;
+                        const int j = tile_of(qi, i);
+                        // O += P V once softmax qi has written P (and rescaled O)
+                        ok = pf_wait(b_tile(qi, 1), i & 1, abort_flag) && wait_v(qi, j);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(qi, j, i > 0);
+                        if (i + 1 >= n_of(qi)) continue;
+                        // the next S overwrites P: wait for this P V to finish reading it
+                        const int j1 = tile_of(qi, i + 1);
+                        ok = pf_wait(b_tile(qi, 2), i & 1, abort_flag) && wait_k(qi, j1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(qi, j1);
+                    }
+                }
+                // every MMA issued so far completes before tensor memory can be freed
+                umma_commit(bar(kPfBarDrain));
+                mbar_wait(bar(kPfBarDrain), 0);
+            }
+            __syncwarp();
+        } else {
+            // ====== softmax: warps 2..5 run slot 0, warps 6..9 slot 1; thread = row = TMEM lane ======
+            const int qi = (warp - kPfSoftmax0) / 4;
+            const int quad = warp & 3;  // a warp reaches TMEM lanes 32 * (warp % 4) .. + 31
+            const int r = quad * 32 + lane;
+            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+            const uint32_t tS = tmem + qi * kPfN + lane_base, tO = tmem + kPfColO + qi * kPfD + lane_base;
+            const uint32_t b_sfull = bar(kPfBarTile + kPfTileBars * qi + 0);
+            const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 1);
+            const uint32_t b_odone = bar(kPfBarTile + kPfTileBars * qi + 2);
+            const int tq = t0 + (split ? 0 : qi) * TOK;  // first chunk token of this slot's queries
+            const int n_mine = split ? (n_tiles - qi + 1) / 2 : n_tiles;  // K/V tiles of this slot
+            const int rows_valid = max(0, min(TOK, q_len - tq));
+            // warps whose 32 rows hold no chunk token only keep the barrier protocol
+            const bool active = (quad * 32) / G < rows_valid;
+            const int tok = min(tq + r / G, q_len - 1);  // rows past the chunk reuse the last token's limit
+            const int pos = o + tok;                      // causal limit: keys 0..pos
+            float m_ref = -CUDART_INF_F, l_sum = 0.f;
+            bool ok = qi < n_slots;
+            for (int i = 0; i < n_mine && ok; ++i) {
+                const int j = split ? 2 * i + qi : i;  // K/V tile
+                ok = __all_sync(0xffffffffu, pf_wait(b_sfull, i & 1, abort_flag));
+                if (!ok) break;
+                if (active) {
+                    tc_fence_after();
+                    // Scores in two 64-key halves a (keys 0..63) and b (64..127), raw q.k; the
+                    // scale (> 0) is applied inside the exponent. Half a is exponentiated
+                    // against the reference max as it stands after a, and its P goes over
+                    // S columns 0..31 (already read). If half b then raises that max (rare
+                    // once a row has warmed up), P of a and its sum are scaled down to the
+                    // new max. P of b goes over columns 32..63.
+                    const int key0 = j * kPfN;
+                    const bool edge = key0 + kPfN - 1 > pos;
+                    const float sl2 = prm.scale_log2;
+                    float h[64];
+                    auto load_half = [&](int half) {  // scores of keys key0 + 64*half .. + 63, masked
+                        tmem_ld64(tS + 64 * half, h);
+                        if (edge) {
+    #pragma unroll
+                            for (int i = 0; i < 64; ++i)
+                                if (key0 + 64 * half + i > pos) h[i] = -CUDART_INF_F;
+                        }
+                    };
+                    auto half_max = [&]() -> float {
+                        float m8[8];
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i) m8[i] = h[i];
+    #pragma unroll
+                        for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], h[i]);
+                        return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+                    };
+                    auto raise = [&](float mx) -> float {  // lazy: move the max only past a 2^8 margin
+                        if (!(mx > m_ref + 8.f)) return 1.f;
+                        const float f = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
+                        m_ref = mx;
+                        return f;
+                    };
+                    auto exp_half = [&](f32x2 (&sum)[4], uint32_t col) {
+                        // no unmasked key yet (m = -inf): every p is 0
+                        pf_exp_half(h, sl2, m_ref == -CUDART_INF_F ? -CUDART_INF_F : -m_ref, sum, tS + col);
+                    };
+                    f32x2 acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc[4] = {0ull, 0ull, 0ull, 0ull};
+                    load_half(0);
+                    float alpha = raise(half_max());  // factor for O and l of the earlier tiles
+                    exp_half(acc_a, 0);
+                    load_half(1);
+                    const float beta = raise(half_max());  // factor for half a of this tile
+                    if (__any_sync(0xffffffffu, beta != 1.f)) {
+                        float pa[32];
+                        tmem_ld32(tS, pa);
+    #pragma unroll
+                        for (int w = 0; w < 32; ++w) {
+                            const uint32_t u = __float_as_uint(pa[w]);
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(u << 16) * beta,
+                                                                            __uint_as_float(u & 0xffff0000u) * beta);
+                            pa[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
+                        }
+                        tmem_st32(tS, pa);
+                        const f32x2 b2 = pack2(beta, beta);
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) mul2(acc_a[e], b2);
+                        alpha *= beta;
+                    }
+                    exp_half(acc, 32);
+                    // O of the earlier tiles takes the same factor as l. S of this tile is
+                    // complete, and so is every earlier MMA (the P V of tile j-1
+                    // included), so O is stable here.
+                    if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
+    #pragma unroll 1
+                        for (int ch = 0; ch < kPfD / 32; ++ch) {
+                            float v[32];
+                            tmem_ld32(tO + ch * 32, v);
+    #pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                            tmem_st32(tO + ch * 32, v);
+                        }
+                    }
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) add2(acc[e], acc_a[e]);
+                    add2(acc[0], acc[1]);
+                    add2(acc[2], acc[3]);
+                    add2(acc[0], acc[2]);
+                    float lo, hi;
+                    unpack2(acc[0], lo, hi);
+                    l_sum = l_sum * alpha + (lo + hi);
+                    tc_fence_before();  // P and O visible to the MMA issued after the barrier
+                }
+                mbar_arrive(b_pready);
+            }
+            // ---- epilogue: out = O / l for the valid rows; a split CTA first merges slot 1 ----
+            if (ok && active) ok = __all_sync(0xffffffffu, pf_wait(b_odone, (n_mine - 1) & 1, abort_flag));
+            float wa = 1.f, wb = 0.f;  // weights of this slot's and of slot 1's (O, l)
+            if (split) {
+                // slot 1 hands (m, l) to slot 0 through shared memory; its O stays in TMEM,
+                // where slot 0's warps (same TMEM lanes) read it. All 8 softmax warps meet here.
+                float *ml = reinterpret_cast<float *>(base + kPfOffML);
+                if (qi == 1) {
+                    ml[r] = m_ref;
+                    ml[kPfM + r] = l_sum;
+                }
+                tc_fence_before();
+                asm volatile("bar.sync 1, %0;" ::"n"(8 * 32) : "memory");
                 tc_fence_after();
-                // Scores in two 64-key halves a (keys 0..63) and b (64..127), raw q.k; the
-                // scale (> 0) is applied inside the exponent. Half a is exponentiated
-                // against the reference max as it stands after a, and its P goes over
-                // S columns 0..31 (already read). If half b then raises that max (rare
-                // once a row has warmed up), P of a and its sum are scaled down to the
-                // new max. P of b goes over columns 32..63.
-                const int key0 = j * kPfN;
-                const bool edge = key0 + kPfN - 1 > pos;
-                const float sl2 = prm.scale_log2;
-                float h[64];
-                auto load_half = [&](int half) {  // scores of keys key0 + 64*half .. + 63, masked
-                    tmem_ld64(tS + 64 * half, h);
-                    if (edge) {
-#pragma unroll
-                        for (int i = 0; i < 64; ++i)
-                            if (key0 + 64 * half + i > pos) h[i] = -CUDART_INF_F;
-                    }
-                };
-                auto half_max = [&]() -> float {
-                    float m8[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) m8[i] = h[i];
-#pragma unroll
-                    for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], h[i]);
-                    return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
-                };
-                auto raise = [&](float mx) -> float {  // lazy: move the max only past a 2^8 margin
-                    if (!(mx > m_ref + 8.f)) return 1.f;
-                    const float f = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
-                    m_ref = mx;
-                    return f;
-                };
-                auto exp_half = [&](f32x2 (&sum)[4], uint32_t col) {
-                    const float nm = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-                    const float sc = m_ref == -CUDART_INF_F ? 0.f : sl2;
-                    pf_exp_half(h, sc, nm, sum, tS + col);
-                };
-                f32x2 acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc[4] = {0ull, 0ull, 0ull, 0ull};
-                load_half(0);
-                float alpha = raise(half_max());  // factor for O and l of the earlier tiles
-                exp_half(acc_a, 0);
-                load_half(1);
-                const float beta = raise(half_max());  // factor for half a of this tile
-                if (__any_sync(0xffffffffu, beta != 1.f)) {
-                    float pa[32];
-                    tmem_ld32(tS, pa);
-#pragma unroll
-                    for (int w = 0; w < 32; ++w) {
-                        const uint32_t u = __float_as_uint(pa[w]);
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(u << 16) * beta,
-                                                                        __uint_as_float(u & 0xffff0000u) * beta);
-                        pa[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
-                    }
-                    tmem_st32(tS, pa);
-                    const f32x2 b2 = pack2(beta, beta);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) mul2(acc_a[e], b2);
-                    alpha *= beta;
+                if (qi == 0) {
+                    const float mb = ml[r], lb = ml[kPfM + r];
+                    const float mm = fmaxf(m_ref, mb);
+                    wa = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mm);
+                    wb = mb == -CUDART_INF_F ? 0.f : exp2f(mb - mm);
+                    l_sum = wa * l_sum + wb * lb;
                 }
-                exp_half(acc, 32);
-                // O of the earlier tiles takes the same factor as l. S of this tile is
-                // complete, and so is every earlier MMA (the P V of tile j-1
-                // included), so O is stable here.
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
-#pragma unroll 1
-                    for (int ch = 0; ch < kPfD / 32; ++ch) {
-                        float v[32];
-                        tmem_ld32(tO + ch * 32, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                        tmem_st32(tO + ch * 32, v);
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) add2(acc[e], acc_a[e]);
-                add2(acc[0], acc[1]);
-                add2(acc[2], acc[3]);
-                add2(acc[0], acc[2]);
-                float lo, hi;
-                unpack2(acc[0], lo, hi);
-                l_sum = l_sum * alpha + (lo + hi);
-                tc_fence_before();  // P and O visible to the MMA issued after the barrier
             }
-            mbar_arrive(b_pready);
-        }
-        // ---- epilogue: out = O / l for the valid rows ----
-        if (ok && active) {
-            ok = __all_sync(0xffffffffu, pf_wait(b_odone, (n_tiles - 1) & 1, abort_flag));
-            if (ok) {
+            if (ok && active && (qi == 0 || !split)) {
                 tc_fence_after();
                 const bool row_ok = r / G < rows_valid;
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const float ia = wa * inv, ib = wb * inv;
+                const uint32_t tOb = tmem + kPfColO + kPfD + lane_base;  // O of slot 1 (split only)
                 const int orow = row_ok ? q0 + tq + r / G : q0;
                 __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
                                      (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
-#pragma unroll 1
+    #pragma unroll 1
                 for (int ch = 0; ch < kPfD / 32; ++ch) {  // 32 columns at a time bounds registers
                     float v[32];
                     tmem_ld32(tO + ch * 32, v);
-#pragma unroll
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= ia;
+                    if (split) {
+                        float vb[32];
+                        tmem_ld32(tOb + ch * 32, vb);
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = fmaf(vb[i], ib, v[i]);
+                    }
+    #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         uint4 pkt;
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i] * inv, v[i + 1] * inv);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[i + 2] * inv, v[i + 3] * inv);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[i + 4] * inv, v[i + 5] * inv);
-                        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[i + 6] * inv, v[i + 7] * inv);
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i], v[i + 1]);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[i + 2], v[i + 3]);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[i + 4], v[i + 5]);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[i + 6], v[i + 7]);
                         pkt.x = *reinterpret_cast<uint32_t *>(&h0);
                         pkt.y = *reinterpret_cast<uint32_t *>(&h1);
                         pkt.z = *reinterpret_cast<uint32_t *>(&h2);
@@ -601,9 +702,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
             }
+            tc_fence_before();
         }
-        tc_fence_before();
-    }
+    };
+    if (split_cta)
+        roles(PfSplit<true>{});
+    else
+        roles(PfSplit<false>{});
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -630,12 +735,14 @@ int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cach
             return PA_ERR_CUDA;
         attr_done[dev] = true;
     }
-    const int n_ct = (max_q_len + kPfNQ * TOK - 1) / (kPfNQ * TOK);
+    const long long slots = static_cast<long long>(num_q_tokens) / (kPfNQ * TOK) + num_seqs;
+    if (slots * s->num_kv_heads > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    (void)max_q_len;  // the slot grid covers every chunk whatever its length
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n_ct, s->num_kv_heads, num_seqs);
+    cfg.gridDim = dim3(static_cast<unsigned>(slots * s->num_kv_heads), 1, 1);
     cfg.blockDim = dim3(kPfThreads);
     cfg.dynamicSmemBytes = kPfSmem;
     cfg.stream = st;
@@ -648,7 +755,7 @@ inline int launch_prefill(void *out, const void *q, const void *k_cache, const v
                           const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *cu_q_lens,
                           const int32_t *context_lens, int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens,
                           float scale, const pa_shape *s, cudaStream_t st) {
-    if (num_seqs > 65535 || s->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs < 1) return PA_ERR_INVALID_ARGUMENT;
     PrefillParams prm{};
     prm.out = out;
     prm.block_tables = block_tables;
@@ -659,6 +766,7 @@ inline int launch_prefill(void *out, const void *q, const void *k_cache, const v
     prm.num_heads = s->num_heads;
     prm.num_kv_heads = s->num_kv_heads;
     prm.num_q_tokens = num_q_tokens;
+    prm.num_seqs = num_seqs;
     prm.scale_log2 = scale * 1.4426950408889634f;
     switch (s->num_heads / s->num_kv_heads) {
         case 1: return launch_prefill_g<1>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);

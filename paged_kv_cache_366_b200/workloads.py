@@ -333,6 +333,18 @@ def prefill_chunk(seed: int = 4, keep_logical: bool = False) -> PagedCase:
                      head_dim=128, dtype="bf16", keep_logical=keep_logical)
 
 
+def spec_verify(seed: int = 5, keep_logical: bool = False) -> PagedCase:
+    """64 sequences each verifying a chunk of 4 tokens (3 drafted + 1), the decode batch's shape otherwise.
+
+    Lengths U{128..2048} after the append, 32/8 heads, head_dim 128, bf16,
+    256 new tokens in all.
+    """
+    rng = np.random.default_rng([seed, _STREAM_LENGTHS])
+    ctx = rng.integers(128, 2048, size=64, endpoint=True)
+    return make_case("spec_verify", seed, context_lens=ctx, q_lens=np.full(64, 4, np.int64), num_heads=32,
+                     num_kv_heads=8, head_dim=128, dtype="bf16", keep_logical=keep_logical)
+
+
 CONFIGS = {
     "tiny": tiny,
     "decode_batch": decode_batch,
@@ -340,4 +352,5 @@ CONFIGS = {
     "prefix_sharing": prefix_sharing,
     "mixed_step": mixed_step,
     "prefill_chunk": prefill_chunk,
+    "spec_verify": spec_verify,
 }
