@@ -180,11 +180,15 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
  * length is q_len = cu_q_lens[b+1] - cu_q_lens[b] and its offset is
  * o = context_lens[b] - q_len. Row j of the chunk sits at absolute position
  * o + j and attends to keys 0 .. o + j (inclusive) of the paged context.
+ * Chunks of any length mix in one call: a decode token is a chunk of 1, a
+ * speculative verify step a chunk of a few tokens, q_len = 0 a sequence with
+ * nothing to attend this step. A whole continuous-batching step is one launch.
  *
  *   out, q       : [num_q_tokens][H][D] device, num_q_tokens = cu_q_lens[B]
  *   cu_q_lens    : int32 [B + 1] device, non-decreasing, cu_q_lens[0] = 0
  *   context_lens : int32 [B] device, >= q_len
- *   max_q_len    : host-side upper bound of every q_len (sizes the grid)
+ *   max_q_len    : host-side upper bound of every q_len (checked, >= 0; the
+ *                  grid is sized from num_q_tokens and num_seqs)
  *   scale        : softmax scale, > 0 (PA_ERR_INVALID_ARGUMENT otherwise)
  * bf16 only, D = 128 only. Runs on the tcgen05 tensor cores with fp32
  * accumulation in tensor memory. Probabilities enter P.V rounded to bf16;
