@@ -135,9 +135,10 @@ def profiled_traffic(workload):
         kv = {}
         with open(path) as f:
             for line in f:
-                if ":" in line and line.lstrip().startswith(("traffic_bytes_per_launch", "source_sha256")):
-                    k, v = line.split(":", 1)
-                    kv[k.strip().strip("-* `")] = v.strip().strip("` ")
+                item = line.strip().lstrip("-* `")  # markdown list items: "- key: value"
+                if ":" in item and item.startswith(("traffic_bytes_per_launch", "source_sha256")):
+                    k, v = item.split(":", 1)
+                    kv[k.strip().strip("`")] = v.strip().strip("` ")
         if kv.get("source_sha256") == decode_source_sha():
             return float(kv["traffic_bytes_per_launch"])
     except Exception:

@@ -120,6 +120,21 @@ def test_bench_step_bytes_and_split():
     assert bench.prefill_flops(case, pre) == sum(range(16, 21)) * 8 * 64 * 4
 
 
+def test_bench_reads_profiled_traffic_only_for_matching_sources(tmp_path, monkeypatch):
+    import bench
+    (tmp_path / "profiles").mkdir()
+    sha = bench.decode_source_sha()
+    (tmp_path / "profiles" / "decode_kernel_w.md").write_text(
+        "# summary\n\n- traffic_bytes_per_launch: 123456\n- source_sha256: %s\n" % sha)
+    (tmp_path / "profiles" / "decode_kernel_stale.md").write_text(
+        "- traffic_bytes_per_launch: 7\n- source_sha256: %s\n" % ("0" * 64))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "decode_source_sha", lambda: sha)
+    assert bench.profiled_traffic("w") == 123456.0
+    assert bench.profiled_traffic("stale") is None
+    assert bench.profiled_traffic("missing") is None
+
+
 def test_bench_reference_arm_runs_on_cpu():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
                           "tiny", "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=600)
