@@ -59,6 +59,25 @@ def test_workspace_sizes():
         pa.pa_decode_workspace_bytes(4, 100, 100, s)  # not a multiple of 64
 
 
+def ws_bytes(B, H, P, D=128):
+    n = B * H * P
+    return n * D * 4 + 2 * ((n * 4 + 15) // 16 * 16)
+
+
+def test_automatic_partitions():
+    # no GPU here, so the policy assumes 148 SMs: 444 resident decode CTAs at 4 query heads per KV head
+    from paged_kv_cache_366_b200 import pa
+    s = shape()
+    # 256 x 8 units fill the GPU four times over: contexts are not split
+    assert pa.pa_decode_workspace_bytes(256, 2016, 0, s) == 0
+    # 64 x 8 units: 512-token partitions (4 of them for 2048 tokens)
+    assert pa.pa_decode_workspace_bytes(64, 2048, 0, s) == ws_bytes(64, 32, 4)
+    # 8 x 8 units of 32 K tokens: 1024-token partitions (32)
+    assert pa.pa_decode_workspace_bytes(8, 32768, 0, s) == ws_bytes(8, 32, 32)
+    # one sequence of 4096 tokens: partitions shrink to 128 so the grid covers the GPU
+    assert pa.pa_decode_workspace_bytes(1, 4096, 0, s) == ws_bytes(1, 32, 32)
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(block_size=32), -2), (dict(head_dim=96), -2), (dict(num_heads=24, num_kv_heads=8), -2),
     (dict(num_heads=30, num_kv_heads=8), -1), (dict(dtype=7), -2), (dict(num_blocks=0), -1),
