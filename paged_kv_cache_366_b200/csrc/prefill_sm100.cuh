@@ -231,6 +231,13 @@ struct PrefillParams {
     float scale_log2;
 };
 
+// max(a, b, c) in one instruction (sm_100 has a three-input max)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // p = 2^(x * sc + nm) for 64 scores of one row: the fp32 p are summed into acc
 // in packed pairs, and the bf16 pairs (keys 2w, 2w+1 in column w) are stored to
 // 32 TMEM columns at taddr.
@@ -239,7 +246,10 @@ __device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, floa
     float pv[32];
 #pragma unroll
     for (int w = 0; w < 32; ++w) {
-        const float a0 = fmaf(x[2 * w], sc, nm), a1 = fmaf(x[2 * w + 1], sc, nm);
+        f32x2 arg = pack2(nm, nm);  // x * sc + nm for the pair, one packed FMA
+        fma2(arg, pack2(x[2 * w], x[2 * w + 1]), pack2(sc, sc));
+        float a0, a1;
+        unpack2(arg, a0, a1);
         const float p0 = ex2_approx(a0);
         const float p1 = ex2_approx(a1);
         add2(acc[w & 3], pack2(p0, p1));
@@ -470,7 +480,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 auto issue_qk = [&](int qi, int j) {  // S_qi = Q K_j^T
                     const uint32_t qb = base_s + kPfOffQ + (split ? 0 : qi) * kPfQTile;
                     const uint32_t kb = base_s + kPfOffK + (j % kPfNSK) * kPfKVTile;
-    #pragma unroll
+#pragma unroll
                     for (int kk = 0; kk < kPfD / 16; ++kk) {
                         umma_bf16(tmem + qi * kPfN,
                                   smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
@@ -483,7 +493,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 auto issue_pv = [&](int qi, int j, bool acc) {  // O_qi (+)= P_qi V_j, P read from tensor memory
                     const uint32_t pt = tmem + qi * kPfN + kPfColP;
                     const uint32_t vb = base_s + kPfOffV + (j % kPfNSV) * kPfKVTile;
-    #pragma unroll
+#pragma unroll
                     for (int kk = 0; kk < kPfN / 16; ++kk) {  // 16 keys = 8 columns of P
                         umma_bf16_ts(tmem + kPfColO + qi * kPfD, pt + kk * 8,
                                      smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV,
@@ -572,19 +582,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     auto load_half = [&](int half) {  // scores of keys key0 + 64*half .. + 63, masked
                         tmem_ld64(tS + 64 * half, h);
                         if (edge) {
-    #pragma unroll
+#pragma unroll
                             for (int i = 0; i < 64; ++i)
                                 if (key0 + 64 * half + i > pos) h[i] = -CUDART_INF_F;
                         }
                     };
-                    auto half_max = [&]() -> float {
+                    auto half_max = [&]() -> float {  // three-input max: two new scores per instruction
                         float m8[8];
-    #pragma unroll
-                        for (int i = 0; i < 8; ++i) m8[i] = h[i];
-    #pragma unroll
-                        for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], h[i]);
-                        return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(h[i], h[i + 8]);
+#pragma unroll
+                        for (int i = 16; i < 64; i += 16)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], h[i + k], h[i + 8 + k]);
+                        return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) *
+                               sl2;
                     };
                     auto raise = [&](float mx) -> float {  // lazy: move the max only past a 2^8 margin
                         if (!(mx > m_ref + 8.f)) return 1.f;
@@ -605,7 +617,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     if (__any_sync(0xffffffffu, beta != 1.f)) {
                         float pa[32];
                         tmem_ld32(tS, pa);
-    #pragma unroll
+#pragma unroll
                         for (int w = 0; w < 32; ++w) {
                             const uint32_t u = __float_as_uint(pa[w]);
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(u << 16) * beta,
@@ -614,7 +626,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         }
                         tmem_st32(tS, pa);
                         const f32x2 b2 = pack2(beta, beta);
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 4; ++e) mul2(acc_a[e], b2);
                         alpha *= beta;
                     }
@@ -623,16 +635,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     // complete, and so is every earlier MMA (the P V of tile j-1
                     // included), so O is stable here.
                     if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {  // tcgen05.ld/st are warp-collective
-    #pragma unroll 1
+#pragma unroll 1
                         for (int ch = 0; ch < kPfD / 32; ++ch) {
                             float v[32];
                             tmem_ld32(tO + ch * 32, v);
-    #pragma unroll
+#pragma unroll
                             for (int i = 0; i < 32; ++i) v[i] *= alpha;
                             tmem_st32(tO + ch * 32, v);
                         }
                     }
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 4; ++e) add2(acc[e], acc_a[e]);
                     add2(acc[0], acc[1]);
                     add2(acc[2], acc[3]);
@@ -675,19 +687,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 const int orow = row_ok ? q0 + tq + r / G : q0;
                 __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(prm.out) +
                                      (static_cast<size_t>(orow) * prm.num_heads + hk * G + r % G) * kPfD;
-    #pragma unroll 1
+#pragma unroll 1
                 for (int ch = 0; ch < kPfD / 32; ++ch) {  // 32 columns at a time bounds registers
                     float v[32];
                     tmem_ld32(tO + ch * 32, v);
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= ia;
                     if (split) {
                         float vb[32];
                         tmem_ld32(tOb + ch * 32, vb);
-    #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = fmaf(vb[i], ib, v[i]);
                     }
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         uint4 pkt;
                         __nv_bfloat162 h0 = __floats2bfloat162_rn(v[i], v[i + 1]);
