@@ -52,6 +52,8 @@
 
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "pa_common.cuh"
 #include "tmap.cuh"
 
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_init(bar(kPfBarDrain), 1);
         for (int qi = 0; qi < kPfNQ; ++qi) {
             mbar_init(bar(kPfBarTile + kPfTileBars * qi + 0), 1);    // sfull: MMA commit
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // pready: every softmax thread
+            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // pready: every softmax thread of the slot
             mbar_init(bar(kPfBarTile + kPfTileBars * qi + 2), 1);    // odone: MMA commit
         }
         *abort_flag = 0;
@@ -738,14 +740,16 @@ int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cach
         !encode_3d(&tm_k, k_cache, kPfD, s->num_kv_heads, rows, 2, 64, 1, kBlockSize, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_3d(&tm_v, v_cache, kPfD, s->num_kv_heads, rows, 2, 64, 1, kBlockSize, CU_TENSOR_MAP_SWIZZLE_128B))
         return PA_ERR_UNSUPPORTED;
-    static bool attr_done[64] = {false};
+    // the shared-memory opt-in, once per device (bit per device; safe across host threads)
+    static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    const uint64_t bit = uint64_t{1} << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
         if (cudaFuncSetAttribute(prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem) !=
             cudaSuccess)
             return PA_ERR_CUDA;
-        attr_done[dev] = true;
+        attr_done.fetch_or(bit, std::memory_order_acq_rel);
     }
     const long long slots = static_cast<long long>(num_q_tokens) / (kPfNQ * TOK) + num_seqs;
     if (slots * s->num_kv_heads > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
