@@ -236,27 +236,37 @@ def barrier():
 # ---------------------------------------------------------------------------
 # CPU oracle: the cpu_baseline leg and the reference arm
 
+def oracle_sample_seqs(case):
+    """Sequences the oracle samples: the decode sequences, or every sequence of a chunk-only workload."""
+    dec, _ = split_seqs(case)
+    return dec if len(dec) else np.arange(case.num_seqs)
+
+
 def oracle_step(case, seqs, num_threads):
-    """The oracle on the step for the listed decode sequences: cache write of their tokens, then decode."""
+    """The oracle on the listed sequences: cache write of all their new tokens, then decode of each
+    sequence's last token (the query that attends to its whole context)."""
     import oracle
+    written = np.concatenate([np.arange(int(case.cu_q_lens[b]), int(case.cu_q_lens[b + 1])) for b in seqs])
     rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in seqs], dtype=np.int64)
-    kc, vc = oracle.reshape_and_cache(case.k_new[rows], case.v_new[rows], case.k_cache, case.v_cache,
-                                      case.slot_mapping[rows])
+    kc, vc = oracle.reshape_and_cache(case.k_new[written], case.v_new[written], case.k_cache, case.v_cache,
+                                      case.slot_mapping[written])
     oracle.decode(case.q[rows], kc, vc, case.block_tables[seqs], case.context_lens[seqs], case.scale,
                   num_threads=num_threads)
 
 
 def step_bytes_for(case, seqs):
+    """Algorithmic bytes of oracle_step on these sequences: the write, then one decode query each."""
     E, H, Hk, D = case.elem_bytes, case.num_heads, case.num_kv_heads, case.head_dim
     ctx = case.context_lens[seqs].astype(np.int64)
     n = len(seqs)
-    return (n * Hk * D * E * 4 + n * 8 + int(ctx.sum()) * Hk * D * E * 2 + n * H * D * E * 2 +
+    t = int(case.q_lens[seqs].astype(np.int64).sum())  # tokens written
+    return (t * Hk * D * E * 4 + t * 8 + int(ctx.sum()) * Hk * D * E * 2 + n * H * D * E * 2 +
             int(((ctx + 15) // 16).sum()) * 4 + 4 * n)
 
 
 def time_oracle(case, budget_s, min_reps=1):
     """Oracle throughput on a bounded sample of the workload's decode sequences; returns a dict."""
-    dec, _ = split_seqs(case)
+    dec = oracle_sample_seqs(case)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     t0 = time.perf_counter()
     oracle_step(case, dec[:1], cores)
@@ -273,7 +283,7 @@ def time_oracle(case, budget_s, min_reps=1):
             break
     nbytes = step_bytes_for(case, seqs) * reps
     return {"value": nbytes / spent / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": "fp64 C oracle (OpenMP, %d threads): cache write + decode of the first %d of %d decode "
+            "sample": "fp64 C oracle (OpenMP, %d threads): cache write + decode of the first %d of %d sampled "
                       "sequences of %s, %d repetition(s), %.2f s" % (cores, n, len(dec), case.name, reps, spent),
             "seconds": spent}
 
@@ -283,7 +293,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     case = make_workload(args.workload)
-    dec, _ = split_seqs(case)
+    dec = oracle_sample_seqs(case)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     # size each step's sample so warmup + steps fit in about two minutes
     budget = max(0.005, 120.0 / (args.steps + args.warmup))
@@ -303,10 +313,11 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": describe(case, dec, np.array([], np.int64)),
+            "data": "synthetic", "config": describe(case, *split_seqs(case)),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle",
                              "sample": "fp64 C oracle: each step = cache write + decode of the first %d of %d "
-                                       "decode sequences of %s" % (n, len(dec), case.name)},
+                                       "sampled sequences of %s (for chunks: all their tokens written, the "
+                                       "last token's query attended)" % (n, len(dec), case.name)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
