@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 2
+#define PA_ABI_VERSION 3
 #define PA_BLOCK_SIZE 16
 
 typedef enum {
@@ -169,6 +169,26 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
               float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
               const pa_shape *shape, void *stream);
+
+/*
+ * pa_decode_partitions, pa_decode_merge: the two kernels of pa_decode, one
+ * call each. They take exactly pa_decode's arguments, and pa_decode is
+ * pa_decode_partitions followed by pa_decode_merge on the same stream with the
+ * same arguments (bit-identical results). pa_decode_partitions runs the
+ * split-context pass: sequences of one partition write out directly, longer
+ * ones write their partials to the workspace. pa_decode_merge combines those
+ * partials into out; it does nothing when no context is split. Exposed so a
+ * caller can put other work between the two or time each kernel. Errors as
+ * for pa_decode.
+ */
+int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                         int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                         void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream);
+int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
+                    int64_t workspace_bytes, const pa_shape *shape, void *stream);
 
 /*
  * pa_prefill_chunk: causal attention for chunks of query tokens placed at a

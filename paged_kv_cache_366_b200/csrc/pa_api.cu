@@ -127,8 +127,10 @@ int allow_smem(K kernel, int bytes, std::atomic<uint64_t> &done) {
     return PA_OK;
 }
 
+constexpr int kStagePartitions = 1, kStageMerge = 2;
+
 template <typename Tq, typename Tc, int D, int G>
-int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
+int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, int stages) {
     using C = pa::DecodeCfg<Tc, D, G>;
     static std::atomic<uint64_t> smem_done{0};
     int arc = allow_smem(pa::decode_kernel<Tq, Tc, D, G>, C::SMEM, smem_done);
@@ -153,23 +155,25 @@ int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
-    if (e != cudaSuccess) return cuda_fail(e);
-    if (prm.max_parts == 1) return PA_OK;
+    if (stages & kStagePartitions) {
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (prm.max_parts == 1 || !(stages & kStageMerge)) return PA_OK;
     cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
     cfg.blockDim = dim3(G * D);
     cfg.dynamicSmemBytes = 0;
-    e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
 template <typename Tq, typename Tc, int D>
-int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st) {
+int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, int stages) {
     switch (g) {
-        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st);
-        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st);
-        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st);
-        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st);
+        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st, stages);
+        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st, stages);
+        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st, stages);
+        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st, stages);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -237,10 +241,14 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
     return g.ws_bytes;
 }
 
-int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-              int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
-              float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes, const pa_shape *shape,
-              void *stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_stages(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                  int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+                  float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
+                  const pa_shape *shape, void *stream, int stages) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -286,15 +294,47 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     const int G = shape->num_heads / shape->num_kv_heads;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (shape->kv_fp8) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st)
-                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st, stages)
+                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st, stages);
     }
     if (shape->dtype == PA_DTYPE_BF16) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st)
-                                      : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st);
+        return shape->head_dim == 128
+                   ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st, stages)
+                   : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st, stages);
     }
-    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st)
-                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st);
+    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st, stages)
+                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st, stages);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+              float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes, const pa_shape *shape,
+              void *stream) {
+    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
+                         kStagePartitions | kStageMerge);
+}
+
+int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                         int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                         void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream) {
+    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
+                         kStagePartitions);
+}
+
+int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
+                    int64_t workspace_bytes, const pa_shape *shape, void *stream) {
+    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
+                         kStageMerge);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,

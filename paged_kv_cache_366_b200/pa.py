@@ -44,7 +44,7 @@ class PaShape(ctypes.Structure):
 EXPORTED = [
     "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
     "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version", "pa_decode_noalloc",
-    "pa_copy_blocks", "pa_swap_blocks",
+    "pa_copy_blocks", "pa_swap_blocks", "pa_decode_partitions", "pa_decode_merge",
 ]
 
 PA_ERR_SCRATCH_LIMIT = -7
@@ -61,8 +61,9 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_decode_workspace_bytes.argtypes = [I32, I32, I32, SP]
     lib.pa_decode_workspace_bytes.restype = I64
-    lib.pa_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
-    lib.pa_decode.restype = ctypes.c_int
+    for fn in (lib.pa_decode, lib.pa_decode_partitions, lib.pa_decode_merge):
+        fn.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
+        fn.restype = ctypes.c_int
     lib.pa_prefill_chunk.argtypes = [P, P, P, P, P, I32, P, P, I32, I32, I32, F, SP, P]
     lib.pa_prefill_chunk.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, SP, P]
@@ -183,7 +184,7 @@ def pa_decode_workspace_bytes(num_seqs: int, max_context_len: int, partition_tok
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
               partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-              k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+              k_scale: float = 0.0, v_scale: float = 0.0, _fn: str = "pa_decode") -> None:
     """Decode attention of one query token per sequence over its paged context."""
     _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
@@ -193,10 +194,21 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
     shape = shape_of(k_cache, H, k_scale, v_scale)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check("pa_decode",
-           lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                         block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
-                         int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape), _stream(stream)))
+    _check(_fn,
+           getattr(lib, _fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                             block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
+                             int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape),
+                             _stream(stream)))
+
+
+def pa_decode_partitions(*args, **kw) -> None:
+    """pa_decode's split-context pass alone (same arguments); pa_decode_merge completes it."""
+    pa_decode(*args, _fn="pa_decode_partitions", **kw)
+
+
+def pa_decode_merge(*args, **kw) -> None:
+    """pa_decode's merge of the split-context partials (same arguments as pa_decode)."""
+    pa_decode(*args, _fn="pa_decode_merge", **kw)
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,

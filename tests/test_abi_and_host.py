@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_messages():
     from paged_kv_cache_366_b200 import pa
-    assert pa.pa_abi_version() == 2
+    assert pa.pa_abi_version() == 3
     assert pa.pa_strerror(0) == "ok"
     assert "workspace" in pa.pa_strerror(-4)
     assert pa.pa_strerror(-99) == "unknown error"
@@ -103,8 +103,8 @@ def test_fp8_cache_shape_validation(kw, code):
 def test_null_pointers_are_rejected_before_any_launch():
     from paged_kv_cache_366_b200 import pa
     s = shape()
-    rc = pa.lib.pa_decode(None, None, None, None, None, 4, None, 2, 64, 1.0, 0, None, 0, ctypes.byref(s), None)
-    assert rc == -1
+    for fn in (pa.lib.pa_decode, pa.lib.pa_decode_partitions, pa.lib.pa_decode_merge):
+        assert fn(None, None, None, None, None, 4, None, 2, 64, 1.0, 0, None, 0, ctypes.byref(s), None) == -1
     rc = pa.lib.pa_reshape_and_cache(None, None, None, None, None, 3, ctypes.byref(s), None)
     assert rc == -1
     assert pa.lib.pa_reshape_and_cache(None, None, None, None, None, 0, ctypes.byref(s), None) == 0

@@ -175,3 +175,23 @@ def test_graph_capture_replays_step(pa):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
     assert pa.pa_get_status() == 0
+
+
+@pytest.mark.parametrize("name", ["decode_batch", "long_context"])
+def test_partitions_then_merge_equals_pa_decode(pa, name):
+    # pa_decode is the two kernels in order: calling them one by one gives the same bits
+    case = W.CONFIGS[name]()
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    mx = int(case.context_lens.max())
+    shape = pa.shape_of(d.k_cache, case.num_heads)
+    ws = torch.empty(max(pa.pa_decode_workspace_bytes(case.num_seqs, mx, 0, shape), 16), dtype=torch.uint8,
+                     device="cuda")
+    args = (d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, 0, ws)
+    whole, parts = torch.empty_like(d.q), torch.empty_like(d.q)
+    pa.pa_decode(whole, *args)
+    pa.pa_decode_partitions(parts, *args)
+    pa.pa_decode_merge(parts, *args)
+    torch.cuda.synchronize()
+    assert pa.pa_get_status() == 0
+    assert torch.equal(whole.view(torch.int16), parts.view(torch.int16))
