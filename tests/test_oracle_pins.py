@@ -445,3 +445,17 @@ def test_block_copy_rejects_indices_outside_the_pool():
     case = small_decode_case(201)
     with pytest.raises(oracle.OracleError):
         oracle.copy_blocks(case.k_cache, case.v_cache, [[0, case.num_blocks]])
+
+
+def test_varlen_batch_matches_library_per_sequence():
+    # one batch mixing a sequence with no new tokens, decode tokens, verify chunks and a
+    # long chunk (the shape a continuous-batching step hands to one launch): every row
+    # equals the library's masked attention for its own sequence, whatever its neighbours
+    case = W.make_case("pin_varlen", 171, context_lens=[9, 40, 3, 130, 77, 200, 1], q_lens=[0, 1, 3, 4, 77, 37, 1],
+                       num_heads=8, num_kv_heads=2, head_dim=64, dtype="f32", scale=0.29, keep_logical=True,
+                       table_slack=1)
+    kc, vc = written(case)
+    got = oracle.prefill(case.q, kc, vc, case.block_tables, case.cu_q_lens, case.context_lens, case.scale)
+    ref = sdpa_prefill(case)
+    assert got.shape == ref.shape == (int(case.q_lens.sum()), 8, 64)
+    assert np.abs(got - ref).max() <= 1e-12
