@@ -182,10 +182,8 @@ def pa_decode_workspace_bytes(num_seqs: int, max_context_len: int, partition_tok
     return int(n)
 
 
-def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
-              partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-              k_scale: float = 0.0, v_scale: float = 0.0, _fn: str = "pa_decode") -> None:
-    """Decode attention of one query token per sequence over its paged context."""
+def _decode(fn: str, out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale) -> None:
     _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(context_lens, torch.int32, "context_lens")
@@ -194,21 +192,35 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
     shape = shape_of(k_cache, H, k_scale, v_scale)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(_fn,
-           getattr(lib, _fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                             block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
-                             int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape),
-                             _stream(stream)))
+    _check(fn,
+           getattr(lib, fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                            block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),
+                            int(partition_tokens), _ptr(workspace), ws_bytes, ctypes.byref(shape),
+                            _stream(stream)))
 
 
-def pa_decode_partitions(*args, **kw) -> None:
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+              partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+              k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+    """Decode attention of one query token per sequence over its paged context."""
+    _decode("pa_decode", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale)
+
+
+def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                         scale: float, partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None,
+                         stream=None, k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """pa_decode's split-context pass alone (same arguments); pa_decode_merge completes it."""
-    pa_decode(*args, _fn="pa_decode_partitions", **kw)
+    _decode("pa_decode_partitions", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale)
 
 
-def pa_decode_merge(*args, **kw) -> None:
+def pa_decode_merge(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+                    partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+                    k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """pa_decode's merge of the split-context partials (same arguments as pa_decode)."""
-    pa_decode(*args, _fn="pa_decode_merge", **kw)
+    _decode("pa_decode_merge", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale)
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
