@@ -47,6 +47,7 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
+PREFILL_SOURCES = ["prefill_sm100.cuh", "pa_common.cuh", "tmap.cuh"]
 WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny",
              "copy_blocks", "swap_blocks", "decode_batch_fp8", "varlen_step", "spec_verify"]
 FP8_K_SCALE, FP8_V_SCALE = 0.02, 1.0 / 48.0
@@ -120,17 +121,17 @@ def load_peak(key="hbm_gbs"):
         return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
-def decode_source_sha():
+def decode_source_sha(sources=None):
     h = hashlib.sha256()
-    for n in DECODE_SOURCES:
+    for n in sources or DECODE_SOURCES:
         with open(os.path.join(ROOT, "paged_kv_cache_366_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def profiled_traffic(workload):
-    """dram read+write bytes per decode launch from the committed ncu summary, if it matches the source."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_%s.md" % workload)
+def profiled_traffic(workload, kernel="decode_kernel", sources=None):
+    """dram read+write bytes per launch from the committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
     try:
         kv = {}
         with open(path) as f:
@@ -139,7 +140,7 @@ def profiled_traffic(workload):
                 if ":" in item and item.startswith(("traffic_bytes_per_launch", "source_sha256")):
                     k, v = item.split(":", 1)
                     kv[k.strip().strip("`")] = v.strip().strip("` ")
-        if kv.get("source_sha256") == decode_source_sha():
+        if kv.get("source_sha256") == decode_source_sha(sources):
             return float(kv["traffic_bytes_per_launch"])
     except Exception:
         pass
@@ -648,7 +649,9 @@ def run_ours(args):
         tf = f / t_pre / 1e12
         line["prefill"] = {"flops": f, "us_per_launch": t_pre * 1e6, "tflops": tf,
                            "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s",
-                                        "frac": tf / tpeak, "traffic": None,
+                                        "frac": tf / tpeak,
+                                        "traffic": profiled_traffic(args.workload, "prefill_kernel",
+                                                                    PREFILL_SOURCES),
                                         "kernel": "prefill_kernel (tcgen05)",
                                         "peak_kind": tkind + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}}
         if not len(dec):

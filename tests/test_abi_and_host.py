@@ -148,7 +148,7 @@ def test_bench_reads_profiled_traffic_only_for_matching_sources(tmp_path, monkey
     (tmp_path / "profiles" / "decode_kernel_stale.md").write_text(
         "- traffic_bytes_per_launch: 7\n- source_sha256: %s\n" % ("0" * 64))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "decode_source_sha", lambda: sha)
+    monkeypatch.setattr(bench, "decode_source_sha", lambda sources=None: sha)
     assert bench.profiled_traffic("w") == 123456.0
     assert bench.profiled_traffic("stale") is None
     assert bench.profiled_traffic("missing") is None
