@@ -265,14 +265,17 @@ def step_bytes_for(case, seqs):
             int(((ctx + 15) // 16).sum()) * 4 + 4 * n)
 
 
-def time_oracle(case, budget_s, min_reps=1):
+def time_oracle(case, budget_s, min_reps=1, threads=None, n_seqs=None):
     """Oracle throughput on a bounded sample of the workload's decode sequences; returns a dict."""
     dec = oracle_sample_seqs(case)
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    t0 = time.perf_counter()
-    oracle_step(case, dec[:1], cores)
-    t_one = max(time.perf_counter() - t0, 1e-4)
-    n = int(max(1, min(len(dec), budget_s / t_one)))
+    cores = threads or (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+    if n_seqs:
+        n = min(len(dec), n_seqs)
+    else:
+        t0 = time.perf_counter()
+        oracle_step(case, dec[:1], cores)
+        t_one = max(time.perf_counter() - t0, 1e-4)
+        n = int(max(1, min(len(dec), budget_s / t_one)))
     seqs = dec[:n]
     reps, spent = 0, 0.0
     while reps < min_reps or spent < budget_s * 0.5:
@@ -286,7 +289,7 @@ def time_oracle(case, budget_s, min_reps=1):
     return {"value": nbytes / spent / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
             "sample": "fp64 C oracle (OpenMP, %d threads): cache write + decode of the first %d of %d sampled "
                       "sequences of %s, %d repetition(s), %.2f s" % (cores, n, len(dec), case.name, reps, spent),
-            "seconds": spent}
+            "seconds": spent, "n_seqs": n}
 
 
 def run_reference(args):
@@ -596,7 +599,11 @@ def run_ours(args):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu = time_oracle(case, args.cpu_seconds)
+        # the same oracle and sample on one thread (one repetition at least)
+        one = time_oracle(case, max(1.0, args.cpu_seconds / 4), threads=1, n_seqs=cpu["n_seqs"])
+        cpu["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1, "sample": one["sample"]}
         cpu.pop("seconds", None)
+        cpu.pop("n_seqs", None)
     parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
     if fp8:
