@@ -600,8 +600,9 @@ def run_ours(args):
     if not args.no_cpu_baseline and world == 1:
         cpu = time_oracle(case, args.cpu_seconds)
         # the same oracle and sample on one thread (one repetition at least)
-        one = time_oracle(case, max(1.0, args.cpu_seconds / 4), threads=1, n_seqs=cpu["n_seqs"])
-        cpu["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1, "sample": one["sample"]}
+        single = time_oracle(case, max(1.0, args.cpu_seconds / 4), threads=1, n_seqs=cpu["n_seqs"])
+        cpu["single_thread"] = {"value": single["value"], "unit": single["unit"], "cores": 1,
+                                "sample": single["sample"]}
         cpu.pop("seconds", None)
         cpu.pop("n_seqs", None)
     parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
