@@ -3,20 +3,23 @@
 
 One step is the whole path for one batch: the KV write of this step's new
 tokens (pa_reshape_and_cache), then paged decode over every decode sequence
-(pa_decode: the split-context kernel, plus the merge kernel when a context
-spans several partitions). The mixed workload also runs the causal prefill
-chunk (pa_prefill_chunk). Inputs are synthetic, seeded and resident in HBM
-before the timed region. Each step is captured once as CUDA graphs and
-replayed between CUDA events on the launching stream. Before every step,
-outside the events, a 256 MiB memset and then a 256 MiB read flush L2 (the
-read makes the memset's dirty lines drain to HBM before the step starts).
+(pa_decode: one kernel, the split-context pass with the merge of split
+contexts fused in). The mixed workload also runs the causal prefill chunk
+(pa_prefill_chunk). Inputs are synthetic, seeded and resident in HBM before
+the timed region. Each step is captured once as CUDA graphs and replayed
+between CUDA events on the launching stream. Before every step, outside the
+events, a 256 MiB memset and then a 256 MiB read flush L2 (the read makes the
+memset's dirty lines drain to HBM before the step starts).
 
 Output: one JSON line on rank 0. `value` is the step's algorithmic bytes
 over the step time, in GB/s and summed over ranks (N > 1 runs independent
 replicas, with no data exchange). `roofline` rates the decode call (its
 algorithmic bytes over its event time) against the measured HBM copy
-bandwidth. `e2e` times the public DecodeStep API from pinned host buffers,
-with the copies inside. `cpu_baseline` is the fp64 oracle on the host cores.
+bandwidth, and against the nominal 8000 GB/s. `e2e` times the public
+DecodeStep API from pinned host buffers, with the copies inside.
+`cpu_baseline` is the fp64 oracle on the host cores. On the decode batch the
+line also carries, under `also`, the long-context decode and the prefill
+chunk, each with its own roofline and clocks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
@@ -148,12 +151,14 @@ def profiled_traffic(workload, kernel="decode_kernel", sources=None):
 
 
 # ---------------------------------------------------------------------------
-# Clock sampling during the timed region
+# Clock sampling during the timed regions
 
 REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
 
 class ClockSampler:
+    """nvidia-smi samples (every 50 ms) of SM clocks and throttle reasons, summarised per time window."""
+
     def __init__(self, gpu: str):
         self.samples = []
         self.proc = None
@@ -185,13 +190,17 @@ class ClockSampler:
         while self.proc and not self.samples and time.time() - t0 < timeout:
             time.sleep(0.05)
 
-    def summary(self, t0, t1):
+    def stop(self):
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            self.proc = None
+
+    def window(self, t0, t1):
+        """Median SM clock, max clock and throttle reasons of the samples taken in [t0, t1]."""
         if not self.samples:
             return None
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
@@ -243,14 +252,16 @@ def oracle_sample_seqs(case):
     return dec if len(dec) else np.arange(case.num_seqs)
 
 
-def oracle_step(case, seqs, num_threads):
+def oracle_step(case, seqs, num_threads, caches=None):
     """The oracle on the listed sequences: cache write of all their new tokens, then decode of each
-    sequence's last token (the query that attends to its whole context)."""
+    sequence's last token (the query that attends to its whole context). With `caches` (writable copies
+    of the pool) the write lands in place, as the GPU's does; otherwise the oracle returns new copies."""
     import oracle
     written = np.concatenate([np.arange(int(case.cu_q_lens[b]), int(case.cu_q_lens[b + 1])) for b in seqs])
     rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in seqs], dtype=np.int64)
-    kc, vc = oracle.reshape_and_cache(case.k_new[written], case.v_new[written], case.k_cache, case.v_cache,
-                                      case.slot_mapping[written])
+    kc, vc = caches if caches is not None else (case.k_cache, case.v_cache)
+    kc, vc = oracle.reshape_and_cache(case.k_new[written], case.v_new[written], kc, vc,
+                                      case.slot_mapping[written], in_place=caches is not None)
     oracle.decode(case.q[rows], kc, vc, case.block_tables[seqs], case.context_lens[seqs], case.scale,
                   num_threads=num_threads)
 
@@ -265,63 +276,74 @@ def step_bytes_for(case, seqs):
             int(((ctx + 15) // 16).sum()) * 4 + 4 * n)
 
 
+def host_cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
 def time_oracle(case, budget_s, min_reps=1, threads=None, n_seqs=None):
     """Oracle throughput on a bounded sample of the workload's decode sequences; returns a dict."""
     dec = oracle_sample_seqs(case)
-    cores = threads or (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+    cores = threads or host_cores()
+    caches = (np.array(case.k_cache, copy=True), np.array(case.v_cache, copy=True))
     if n_seqs:
         n = min(len(dec), n_seqs)
     else:
         t0 = time.perf_counter()
-        oracle_step(case, dec[:1], cores)
+        oracle_step(case, dec[:1], cores, caches)
         t_one = max(time.perf_counter() - t0, 1e-4)
         n = int(max(1, min(len(dec), budget_s / t_one)))
     seqs = dec[:n]
     reps, spent = 0, 0.0
     while reps < min_reps or spent < budget_s * 0.5:
         t0 = time.perf_counter()
-        oracle_step(case, seqs, cores)
+        oracle_step(case, seqs, cores, caches)
         spent += time.perf_counter() - t0
         reps += 1
         if spent > budget_s:
             break
     nbytes = step_bytes_for(case, seqs) * reps
     return {"value": nbytes / spent / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": "fp64 C oracle (OpenMP, %d threads): cache write + decode of the first %d of %d sampled "
+            "sample": "fp64 C oracle (OpenMP, %d threads): cache write (in place) + decode of the first %d of %d "
                       "sequences of %s, %d repetition(s), %.2f s" % (cores, n, len(dec), case.name, reps, spent),
             "seconds": spent, "n_seqs": n}
 
 
 def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step writes the step's new tokens in place
+    and decodes every sampled sequence. All sequences are taken when (warmup + steps) of them fit in
+    about two minutes, else the first n that do."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     case = make_workload(args.workload)
     dec = oracle_sample_seqs(case)
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    # size each step's sample so warmup + steps fit in about two minutes
+    cores = host_cores()
+    caches = (np.array(case.k_cache, copy=True), np.array(case.v_cache, copy=True))
     budget = max(0.005, 120.0 / (args.steps + args.warmup))
     t0 = time.perf_counter()
-    oracle_step(case, dec[:1], cores)
-    t_one = max(time.perf_counter() - t0, 1e-4)
-    n = int(max(1, min(len(dec), budget / t_one)))
+    oracle_step(case, dec, cores, caches)
+    t_all = max(time.perf_counter() - t0, 1e-4)
+    n = len(dec) if t_all <= budget else int(max(1, len(dec) * budget / t_all))
     seqs = dec[:n]
     for _ in range(args.warmup):
-        oracle_step(case, seqs, cores)
+        oracle_step(case, seqs, cores, caches)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(case, seqs, cores)
+        oracle_step(case, seqs, cores, caches)
     dt = time.perf_counter() - t0
     nbytes = step_bytes_for(case, seqs) * args.steps
     value = nbytes / dt / 1e9
+    config = describe(case, *split_seqs(case))
+    config["sampled_seqs"] = int(n)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": describe(case, *split_seqs(case)),
+            "data": "synthetic", "config": config,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-                             "sample": "fp64 C oracle: each step = cache write + decode of the first %d of %d "
-                                       "sampled sequences of %s (for chunks: all their tokens written, the "
-                                       "last token's query attended)" % (n, len(dec), case.name)},
+                             "sample": "fp64 C oracle: each step = cache write (in place) of the step's new tokens "
+                                       "+ decode of %s%d of %d sequences of %s (for chunks: all their tokens "
+                                       "written, the last token's query attended)" % (
+                                           "all " if n == len(dec) else "the first ", n, len(dec), case.name)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -333,6 +355,7 @@ def run_reference(args):
 # Workloads whose whole attention is one pa_prefill_chunk launch over every
 # sequence (decode tokens as chunks of 1, verify chunks, prefill chunks).
 ONE_LAUNCH = ("varlen_step", "spec_verify")
+NOMINAL_HBM_GBS = 8000.0  # the nominal HBM peak the targets are quoted against
 
 
 def make_workload(name):
@@ -345,20 +368,39 @@ def make_workload(name):
     return W.CONFIGS[name]()
 
 
-def run_ours(args):
+def unique_kv_bytes(case, dec):
+    """K/V bytes of the distinct physical rows the decode sequences read (shared blocks counted once)."""
+    Hk, D, E = case.num_kv_heads, case.head_dim, case.elem_bytes
+    rows = {}
+    for b in dec:
+        c = int(case.context_lens[b])
+        for i in range((c + 15) // 16):
+            pb = int(case.block_tables[b, i])
+            rows[pb] = max(rows.get(pb, 0), min(16, c - 16 * i))
+    return sum(rows.values()) * Hk * D * E * 2
+
+
+class Flush:
+    """Evict L2 between timed steps: write a buffer larger than L2, then read another, so the write's
+    dirty lines reach HBM before the timed events rather than during them."""
+
+    def __init__(self):
+        import torch
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r)
+
+
+def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
+    """Set up one workload on the device, capture its step and parts as CUDA graphs, and time them.
+
+    Returns a dict with the case, the step's algorithmic bytes by part, the summed step time (seconds over
+    `steps` steps), the per-part times per step, clocks during the step loop and the e2e figures."""
     import torch
-    import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.gpus != world and world > 1:
-        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-
     from paged_kv_cache_366_b200 import pa
     from paged_kv_cache_366_b200.step import DecodeStep
 
@@ -367,9 +409,9 @@ def run_ours(args):
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
         return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
-    case = make_workload(args.workload)
+    case = make_workload(name)
     dec, pre = split_seqs(case)
-    fp8 = args.workload == "decode_batch_fp8"
+    fp8 = name == "decode_batch_fp8"
     ks, vs = (FP8_K_SCALE, FP8_V_SCALE) if fp8 else (0.0, 0.0)
     nbytes = step_bytes(case, dec, pre, 1 if fp8 else None)
 
@@ -396,7 +438,7 @@ def run_ours(args):
     max_ctx = int(case.context_lens[dec].max()) if len(dec) else 0
     ws_n = pa.pa_decode_workspace_bytes(len(dec), max_ctx, 0, shape) if len(dec) else 0
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
-    decode_kernels = 2 if ws_n else 1
+    ws_split = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
 
     if len(pre):
         p0, p1 = int(pre[0]), int(pre[-1]) + 1
@@ -411,20 +453,21 @@ def run_ours(args):
     def do_write():
         pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, k_scale=ks, v_scale=vs)
 
-    # pa_decode as its two kernels, so each is timed on its own (same arguments, same result)
-    def do_decode_partitions():
-        pa.pa_decode_partitions(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale,
-                                0, ws, k_scale=ks, v_scale=vs)
+    def do_decode():  # one kernel: the split-context pass with the merge fused in
+        pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws,
+                     k_scale=ks, v_scale=vs)
 
-    def do_merge():
-        pa.pa_decode_merge(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0,
-                           ws, k_scale=ks, v_scale=vs)
+    out_split = torch.empty_like(q_dec) if len(dec) else None
+
+    def do_partitions():  # the split-context pass alone, without the merge (not part of the step)
+        pa.pa_decode_partitions(out_split, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx,
+                                case.scale, 0, ws_split, k_scale=ks, v_scale=vs)
 
     def do_prefill():
         pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
                             case.scale)
 
-    one = args.workload in ONE_LAUNCH
+    one = name in ONE_LAUNCH
     out_all = torch.empty_like(q)
     max_q_all = int(case.q_lens.max())
 
@@ -432,25 +475,25 @@ def run_ours(args):
         pa.pa_prefill_chunk(out_all, q, k_cache, v_cache, tables, cu, lens, max_q_all, case.scale)
 
     parts = [("write", do_write)]
+    extra = []
     if one:
         parts.append(("attention", do_all))
-        launches_per_step = 2
     else:
         if len(pre):
             parts.append(("prefill", do_prefill))
         if len(dec):
-            parts.append(("decode", do_decode_partitions))
-            if ws_n:  # some context is split: the merge kernel follows
-                parts.append(("merge", do_merge))
-        launches_per_step = 1 + (1 if len(pre) else 0) + (decode_kernels if len(dec) else 0)
+            parts.append(("decode", do_decode))
+            if ws_n:
+                extra.append(("partitions_only", do_partitions))
+    launches_per_step = len(parts)
 
     # one graph for the whole step (the headline), one per part (breakdown, roofline)
     graphs = []
     with torch.cuda.stream(stream):
-        for _, fn in parts:  # eager once, then capture
+        for _, fn in parts + extra:  # eager once, then capture
             fn()
         stream.synchronize()
-        for _, fn in parts:
+        for _, fn in parts + extra:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
@@ -462,42 +505,25 @@ def run_ours(args):
     torch.cuda.synchronize()
     status = pa.pa_get_status(stream)
     if status:
-        raise SystemExit("device status 0x%x after the first step" % status)
+        raise SystemExit("device status 0x%x after the first step of %s" % (status, name))
 
-    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-
-    class _Flush:
-        """Evict L2: write a buffer larger than L2, then read another, so the write's
-        dirty lines reach HBM before the timed events rather than during them."""
-
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            torch.sum(flush_r)
-
-    flush = _Flush()
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            flush.zero_()
+        for _ in range(warmup):
+            flush()
             g_step.replay()
-            flush.zero_()
+            flush()
             for g in graphs:
                 g.replay()
     torch.cuda.synchronize()
 
-    # timed region: K steps, each one graph replay between events, L2 flushed before each
-    sampler = ClockSampler(gpu_id_for(local_rank)) if rank == 0 else None
-    if sampler:
-        sampler.wait_ready()
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+    # timed region: `steps` steps, each one graph replay between events, L2 flushed before each
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            flush.zero_()
+        for i in range(steps):
+            flush()
             step_ev[i][0].record(stream)
             g_step.replay()
             step_ev[i][1].record(stream)
@@ -506,61 +532,51 @@ def run_ours(args):
     wall1 = time.time()
     status = pa.pa_get_status(stream)
     if status:
-        raise SystemExit("device status 0x%x after the timed steps" % status)
+        raise SystemExit("device status 0x%x after the timed steps of %s" % (status, name))
     total = sum(a.elapsed_time(b) for a, b in step_ev) * 1e-3
 
     # per-part times (each part its own graph, events between), for the breakdown and rooflines
-    n_parts_steps = min(args.steps, 500)
-    n_ev = len(parts) + 1
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_parts_steps)]
+    n_parts_steps = min(steps, 500)
+    names = [n for n, _ in parts + extra]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(graphs))] for _ in range(n_parts_steps)]
     with torch.cuda.stream(stream):
         for i in range(n_parts_steps):
-            flush.zero_()
-            ev = events[i]
-            ev[0].record(stream)
             for j, g in enumerate(graphs):
+                flush()
+                events[i][2 * j].record(stream)
                 g.replay()
-                ev[j + 1].record(stream)
+                events[i][2 * j + 1].record(stream)
     torch.cuda.synchronize()
-    per_part = {name: 0.0 for name, _ in parts}
-    for ev in events:
-        for j, (name, _) in enumerate(parts):
-            per_part[name] += ev[j].elapsed_time(ev[j + 1]) * 1e-3
-    per_part = {k: v * args.steps / n_parts_steps for k, v in per_part.items()}  # per-step sums as over K steps
-    sum_bytes, t_max = aggregate(float(nbytes["total"]) * args.steps, total)
-    value = sum_bytes / t_max / 1e9
-    ms_per_step = t_max / args.steps * 1e3
+    per_part = {n: sum(ev[2 * j].elapsed_time(ev[2 * j + 1]) for ev in events) * 1e-3 / n_parts_steps
+                for j, n in enumerate(names)}  # seconds per step
+    clocks = sampler.window(wall0, wall1) if sampler else None
 
     # end to end through the public API, host buffers, copies inside (decode workloads)
     e2e = None
-    if len(dec) and not len(pre):
-        hk_cache = k_cache  # the pool is device-resident state
-        step = DecodeStep(hk_cache, v_cache, case.num_heads, len(dec), case.max_blocks_per_seq, max_ctx,
+    if want_e2e and len(dec) and not len(pre):
+        step = DecodeStep(k_cache, v_cache, case.num_heads, len(dec), case.max_blocks_per_seq, max_ctx,
                           case.scale, k_scale=ks, v_scale=vs)
-
         rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)
-        # staged inputs: the step's six inputs live in one pinned buffer (one copy in per step)
-        views = step.inputs()
+        views = step.inputs()  # staged inputs: the step's six inputs in one pinned buffer
 
         def fill(dst, a):
             a = np.ascontiguousarray(a)
             src = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
             (dst.view(torch.int16) if a.dtype == np.uint16 else dst).copy_(src)
-        assert not fp8 or case.dtype == "bf16"
         fill(views["q"], case.q[rows])
         fill(views["k_new"], case.k_new[rows])
         fill(views["v_new"], case.v_new[rows])
         fill(views["slot_mapping"], case.slot_mapping[rows])
         fill(views["block_tables"], case.block_tables[d0:d1])
         fill(views["context_lens"], case.context_lens[d0:d1])
-        n_e2e = max(10, min(args.steps, 500))
-        for _ in range(max(3, args.warmup)):
+        n_e2e = max(10, min(steps, 500))
+        for _ in range(max(3, warmup)):
             step.run()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
         barrier()
         for i in range(n_e2e):
             with torch.cuda.stream(step.stream):
-                flush.zero_()
+                flush()
                 ev[i][0].record(step.stream)
             step.launch()
             with torch.cuda.stream(step.stream):
@@ -570,32 +586,97 @@ def run_ours(args):
         t_e2e = sum(a.elapsed_time(b) for a, b in ev) * 1e-3
         b_e2e, t_e2e = aggregate(float(nbytes["total"]) * n_e2e, t_e2e)
         e2e = {"value": b_e2e / t_e2e / 1e9, "unit": UNIT, "h2d_bytes_per_step": step.h2d_bytes(),
-               "d2h_bytes_per_step": step.d2h_bytes(), "steps": n_e2e,
-               "ms_per_step": t_e2e / n_e2e * 1e3,
+               "d2h_bytes_per_step": step.d2h_bytes(), "steps": n_e2e, "ms_per_step": t_e2e / n_e2e * 1e3,
                "api": "paged_kv_cache_366_b200.step.DecodeStep, staged inputs (one copy in, one out; CUDA graph)"}
+    del graphs, g_step
+    return {"case": case, "dec": dec, "pre": pre, "nbytes": nbytes, "total": total, "per_part": per_part,
+            "clocks": clocks, "e2e": e2e, "one": one, "fp8": fp8, "ks": ks, "vs": vs,
+            "launches_per_step": launches_per_step, "wall": (wall0, wall1)}
+
+
+def decode_roofline(m, peak, peak_kind, name):
+    """Roofline of the dominant decode kernel: decode_kernel with the fused merge (the pa_decode call)."""
+    t_dec = m["per_part"]["decode"]
+    nb = m["nbytes"]["decode"]
+    achieved = nb / t_dec / 1e9
+    r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+         "frac_of_nominal": achieved / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
+         "traffic": profiled_traffic(name), "kernel": "decode_kernel (split-context pass with the merge fused in; "
+                                                      "the whole pa_decode call)",
+         "algorithmic_bytes_per_launch": nb, "us_per_launch": t_dec * 1e6,
+         "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind}
+    if "partitions_only" in m["per_part"]:
+        r["partition_pass_alone_us"] = m["per_part"]["partitions_only"] * 1e6
+    return r
+
+
+def prefill_roofline(m, name):
+    case, pre = m["case"], m["pre"]
+    f = prefill_flops(case, pre)
+    t_pre = m["per_part"]["prefill"]
+    tpeak, tkind = load_peak("bf16_tflops")
+    tf = f / t_pre / 1e12
+    return {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
+            "traffic": profiled_traffic(name, "prefill_kernel", PREFILL_SOURCES), "kernel": "prefill_kernel (tcgen05)",
+            "flops_per_launch": f, "us_per_launch": t_pre * 1e6,
+            "peak_kind": tkind + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    sampler = ClockSampler(gpu_id_for(local_rank)) if rank == 0 else None
+    if sampler:
+        sampler.wait_ready()
+    flush = Flush()
+    m = measure_gpu(args.workload, args.steps, args.warmup, flush, sampler, want_e2e=True)
+    case, dec, pre, nbytes = m["case"], m["dec"], m["pre"], m["nbytes"]
+    sum_bytes, t_max = aggregate(float(nbytes["total"]) * args.steps, m["total"])
+    value = sum_bytes / t_max / 1e9
+    ms_per_step = t_max / args.steps * 1e3
+
+    # companions of the headline in the same run: the other target config of the decode kernel
+    # (long context) and the tensor-core prefill chunk, each with its own roofline and clocks
+    also = {}
+    if not args.no_also and args.workload == "decode_batch":
+        peak, peak_kind = load_peak()
+        for extra in ("long_context", "prefill_chunk"):
+            torch.cuda.empty_cache()
+            steps_x = max(5, min(args.steps, 50))
+            mx = measure_gpu(extra, steps_x, args.warmup, flush, sampler, want_e2e=False)
+            b_x, t_x = aggregate(float(mx["nbytes"]["total"]) * steps_x, mx["total"])
+            ent = {"steps": steps_x, "ms_per_step": t_x / steps_x * 1e3, "value": b_x / t_x / 1e9, "unit": UNIT,
+                   "clocks": mx["clocks"], "config": describe(mx["case"], mx["dec"], mx["pre"])}
+            if len(mx["dec"]):
+                ent["roofline"] = decode_roofline(mx, peak, peak_kind, extra)
+            if len(mx["pre"]):
+                ent["roofline"] = prefill_roofline(mx, extra)
+            also[extra] = ent
+            del mx
 
     if world > 1:
         dist.destroy_process_group()
+    if sampler:
+        sampler.stop()
     if rank != 0:
         return 0
 
-    clocks = sampler.summary(wall0, wall1) if sampler else None
     peak, peak_kind = load_peak()
+    per_part = m["per_part"]
     roof = None
-    if not one and len(dec):
-        # the dominant kernel: decode_kernel (the split-context pass), timed on its own. Its
-        # algorithmic bytes are the whole decode's (K/V, q, out, tables); the merge that
-        # follows reads the partials back from L2 and is reported beside it.
-        t_dec = per_part["decode"] / args.steps
-        t_merge = per_part.get("merge", 0.0) / args.steps
-        achieved = nbytes["decode"] / t_dec / 1e9
-        call = nbytes["decode"] / (t_dec + t_merge) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": profiled_traffic(args.workload), "kernel": "decode_kernel (split-context pass)",
-                "algorithmic_bytes_per_launch": nbytes["decode"], "us_per_launch": t_dec * 1e6,
-                "merge_us_per_launch": t_merge * 1e6,
-                "pa_decode_call": {"achieved": call, "frac": call / peak, "us": (t_dec + t_merge) * 1e6},
-                "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind}
+    if not m["one"] and len(dec):
+        roof = decode_roofline(m, peak, peak_kind, args.workload)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu = time_oracle(case, args.cpu_seconds)
@@ -605,12 +686,13 @@ def run_ours(args):
                                 "sample": single["sample"]}
         cpu.pop("seconds", None)
         cpu.pop("n_seqs", None)
-    parts_ms = {k: v / args.steps * 1e3 for k, v in per_part.items()}
+    parts_ms = {k: v * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
-    if fp8:
-        config.update({"workload": "decode_batch_fp8", "kv_dtype": "fp8_e4m3", "k_scale": ks, "v_scale": vs})
-    config.update({"l2": "flushed before every step, outside the events: 256 MiB memset, then a 256 MiB read "
-                         "so the memset's write-back is not charged to the step",
+    if m["fp8"]:
+        config.update({"workload": "decode_batch_fp8", "kv_dtype": "fp8_e4m3", "k_scale": m["ks"],
+                       "v_scale": m["vs"]})
+    config.update({"l2": "flushed before every step and every timed part, outside the events: 256 MiB memset, "
+                         "then a 256 MiB read so the memset's write-back is not charged to the step",
                    "timing": "one CUDA graph replay per step between CUDA events on the launching stream; "
                              "per-part times from a second loop of per-part graphs",
                    "parallelism": "replicas" if args.gpus > 1 else "single GPU",
@@ -619,18 +701,25 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": case.dtype, "data": "synthetic (seeded; see paged_kv_cache_366_b200/"
                                                                  "workloads.py)",
-            "config": config, "pct_of_hbm_peak": value / peak,
+            "config": config, "pct_of_hbm_peak": value / peak, "pct_of_nominal_peak": value / NOMINAL_HBM_GBS,
             "decode_tokens_per_s": len(dec) * args.gpus / (t_max / args.steps),
             "kv_gbs": nbytes["kv_decode"] * args.gpus / (t_max / args.steps) / 1e9,
-            "ms_per_part": parts_ms, "step_bytes": nbytes, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
-            "wall_s_timed_region": wall1 - wall0}
-    if one:
+            "ms_per_part": parts_ms, "step_bytes": nbytes, "roofline": roof, "cpu_baseline": cpu, "e2e": m["e2e"],
+            "clocks": m["clocks"], "gpu_launches": m["launches_per_step"] * args.steps,
+            "wall_s_timed_region": m["wall"][1] - m["wall"][0]}
+    if args.workload.startswith("prefix_sharing"):
+        ub = unique_kv_bytes(case, dec) + (nbytes["decode"] - nbytes["kv_decode"])
+        t_dec = per_part["decode"]
+        line["unique_bytes"] = {"decode_bytes": ub, "gbs": ub / t_dec / 1e9, "frac": ub / t_dec / 1e9 / peak,
+                                "frac_of_nominal": ub / t_dec / 1e9 / NOMINAL_HBM_GBS,
+                                "note": "K/V bytes of the distinct physical rows read (the shared prefix once), "
+                                        "plus q, out and tables, over the pa_decode time"}
+    if m["one"]:
         # One launch does the decode tokens (HBM-bound) and the chunks (tensor-bound
         # when long). Its floor is the chunks' FLOPs at the bf16 peak plus the decode
         # tokens' bytes at the copy bandwidth; a launch of verify chunks alone is
         # HBM-bound (a few rows per KV head).
-        t_one = per_part["attention"] / args.steps
+        t_one = per_part["attention"]
         tpeak, tkind = load_peak("bf16_tflops")
         f = prefill_flops(case, pre)
         attn_bytes = nbytes["decode"] + nbytes["prefill"]
@@ -649,21 +738,17 @@ def run_ours(args):
                 "floor_us": t_floor * 1e6, "us_per_launch": t_one * 1e6,
                 "peak_kind": "measured (MEASURED_PEAKS.json hbm_gbs%s)" % (
                     "" if not long_chunks else " and bf16_tflops")}
+        if not long_chunks:
+            roof["frac_of_nominal"] = attn_bytes / t_one / 1e9 / NOMINAL_HBM_GBS
         line["roofline"] = roof
-    if not one and len(pre):
-        f = prefill_flops(case, pre)
-        t_pre = per_part["prefill"] / args.steps
-        tpeak, tkind = load_peak("bf16_tflops")
-        tf = f / t_pre / 1e12
-        line["prefill"] = {"flops": f, "us_per_launch": t_pre * 1e6, "tflops": tf,
-                           "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s",
-                                        "frac": tf / tpeak,
-                                        "traffic": profiled_traffic(args.workload, "prefill_kernel",
-                                                                    PREFILL_SOURCES),
-                                        "kernel": "prefill_kernel (tcgen05)",
-                                        "peak_kind": tkind + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}}
+    if not m["one"] and len(pre):
+        pr = prefill_roofline(m, args.workload)
+        line["prefill"] = {"flops": pr["flops_per_launch"], "us_per_launch": pr["us_per_launch"],
+                           "tflops": pr["achieved"], "roofline": pr}
         if not len(dec):
-            line["roofline"] = line["prefill"]["roofline"]
+            line["roofline"] = pr
+    if also:
+        line["also"] = also
     print(json.dumps(line), flush=True)
     return 0
 
@@ -755,6 +840,7 @@ def run_blocks(args):
             b.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
+    sampler.stop()
     t = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
     value = nbytes / t / 1e9
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -765,7 +851,7 @@ def run_blocks(args):
                        "l2": "flushed before every step, outside the events (memset then read)"},
             "roofline": {"bound": bound, "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
                          "traffic": None, "kernel": "copy_blocks_kernel", "peak_kind": peak_note},
-            "cpu_baseline": None, "e2e": None, "clocks": sampler.summary(wall0, wall1),
+            "cpu_baseline": None, "e2e": None, "clocks": sampler.window(wall0, wall1),
             "gpu_launches": launches * args.steps}
     print(json.dumps(line), flush=True)
     return 0
@@ -779,6 +865,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode_batch", choices=WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true", help="skip the long-context and prefill companions")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle timing")
     args = ap.parse_args(argv)
     if args.warmup < 3:

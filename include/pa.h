@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 3
+#define PA_ABI_VERSION 4
 #define PA_BLOCK_SIZE 16
 
 typedef enum {
@@ -79,6 +79,7 @@ typedef enum {
 #define PA_STATUS_BAD_CONTEXT 0x4u    /* context length < 0, > MB * 16, or > max_context_len */
 #define PA_STATUS_WAIT_TIMEOUT 0x8u   /* a bounded wait on an async copy gave up */
 #define PA_STATUS_BAD_QUERY 0x10u     /* prefill: q_len > context_len or cu_q_lens not increasing */
+#define PA_STATUS_BAD_WORKSPACE 0x20u /* pa_decode: a merge ticket had more arrivals than partitions */
 
 typedef struct {
     int32_t num_heads;    /* H, query heads */
@@ -129,8 +130,10 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
 /*
  * pa_decode_workspace_bytes: scratch size pa_decode needs for these sizes
  * and this partition_tokens (0 = automatic), on the current device. It is 0
- * when the single-pass kernel covers every sequence. Negative on bad
- * arguments.
+ * when no context is split across partitions. Negative on bad arguments.
+ * Layout: fp32 partial outputs [B][H][P][D], partial maxima and sums
+ * [B][H][P] each, then 64-bit merge tickets [B][Hk], each part 16-byte
+ * aligned.
  */
 int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int32_t partition_tokens,
                                   const pa_shape *shape);
@@ -156,12 +159,20 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
  *   partition_tokens : 0 = automatic. Otherwise tokens per split-context
  *                  partition, a multiple of 64 and >= 64. A context longer
  *                  than one partition is split. Each partition writes
- *                  (max, sum, unnormalised O) to the workspace and a second
- *                  kernel merges them.
+ *                  (max, sum, unnormalised O) to the workspace; the last
+ *                  partition of a (sequence, KV head) to finish, found by a
+ *                  ticket counter in the workspace, merges them. pa_decode is
+ *                  one kernel launch.
  *   workspace    : device scratch of >= pa_decode_workspace_bytes(...) bytes,
  *                  16-byte aligned. It may be NULL when that size is 0. Its
- *                  contents need no initialisation, and calls that overlap on
- *                  the GPU must not share one.
+ *                  contents need no initialisation: each merge ticket holds a
+ *                  stamp of the call that wrote it (different for every host
+ *                  call, kept by a CUDA graph replay, which leaves its tickets
+ *                  reset), and a ticket with another stamp counts as empty. A
+ *                  ticket with this call's stamp and too many arrivals (two
+ *                  overlapping replays of one graph, say) sets
+ *                  PA_STATUS_BAD_WORKSPACE. Calls that overlap on the GPU must
+ *                  not share a workspace.
  * Accumulation is fp32 whatever the dtype. bf16 output is rounded once, to
  * nearest even.
  */
@@ -171,15 +182,16 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               const pa_shape *shape, void *stream);
 
 /*
- * pa_decode_partitions, pa_decode_merge: the two kernels of pa_decode, one
- * call each. They take exactly pa_decode's arguments, and pa_decode is
- * pa_decode_partitions followed by pa_decode_merge on the same stream with the
- * same arguments (bit-identical results). pa_decode_partitions runs the
- * split-context pass: sequences of one partition write out directly, longer
- * ones write their partials to the workspace. pa_decode_merge combines those
- * partials into out; it does nothing when no context is split. Exposed so a
- * caller can put other work between the two or time each kernel. Errors as
- * for pa_decode.
+ * pa_decode_partitions, pa_decode_merge: pa_decode as two kernels, one call
+ * each. They take exactly pa_decode's arguments, and pa_decode_partitions
+ * followed by pa_decode_merge on the same stream with the same arguments gives
+ * pa_decode's result bit for bit. pa_decode_partitions runs the split-context
+ * pass without the fused merge: sequences of one partition write out
+ * directly, longer ones write their partials to the workspace.
+ * pa_decode_merge combines those partials into out; it does nothing when no
+ * context is split. Neither touches the merge tickets, so the workspace needs
+ * no zeroing for them. Exposed so a caller can put other work between the two
+ * or time each kernel. Errors as for pa_decode.
  */
 int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
                          const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
@@ -271,17 +283,21 @@ int pa_swap_blocks(void *dst, const void *src, const int64_t *block_pairs, int64
  *  - The array is a static device variable. Every GPU on which the library's
  *    module is loaded holds those bytes until the process exits.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current, and caches it. Make that
- *    first call outside any stream capture; later calls only enqueue kernels.
+ *    (cudaGetSymbolAddress) with that device current, and caches it with the
+ *    device's current context. Make that first call outside any stream
+ *    capture. A later call in a different context of that device (after a
+ *    cudaDeviceReset, say) looks the address up again.
  *  - Requests whose partials need more than PA_NOALLOC_SCRATCH_BYTES (see
  *    pa_decode_workspace_bytes) return PA_ERR_SCRATCH_LIMIT and launch nothing.
  *    Use pa_decode with your own workspace for those, or a larger
  *    partition_tokens.
  *  - Every call on a device shares the one array, and the array keeps whatever
- *    the last call left in it. Nothing in it needs to start at zero: each call
- *    writes every partial it later reads. Calls that may overlap on the GPU
- *    (different streams, or different host threads on one device) race on the
- *    array and must be serialized by the caller.
+ *    the last call left in it. Nothing in it needs to start at zero: a call
+ *    runs pa_decode as its two kernels (pa_decode_partitions, then
+ *    pa_decode_merge), and the first writes every partial the second reads.
+ *    Calls that may overlap on the GPU (different streams, or different host
+ *    threads on one device) race on the array and must be serialized by the
+ *    caller.
  * The library calls no cudaMalloc, cudaFree or other allocating routine here.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -294,6 +310,11 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
 /*
  * pa_get_status: synchronize `stream`, copy the device status word of the
  * current device to *status (PA_STATUS_* flags, 0 = clean), then clear it.
+ * There is one status word per device, shared by every stream and host
+ * thread that uses the library on it: the flags read may have been raised by
+ * a call on another stream (and a flag raised by a call still running on
+ * another stream may be cleared before it is read there). Callers that need
+ * per-stream attribution serialize their pa_get_status calls with the work.
  */
 int pa_get_status(uint32_t *status, void *stream);
 

@@ -176,12 +176,22 @@ def prefill(q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, scale: f
     return out
 
 
-def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping):
-    """Return copies of (k_cache, v_cache) with each new token's row written to its slot."""
+def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, in_place: bool = False):
+    """Return copies of (k_cache, v_cache) with each new token's row written to its slot.
+
+    With in_place=True the given arrays (C-contiguous, writable) are written
+    and returned instead of copies.
+    """
     k = _c(k)
     v = _c(v)
-    kc = np.array(k_cache, copy=True, order="C")
-    vc = np.array(v_cache, copy=True, order="C")
+    if in_place:
+        if not (k_cache.flags.c_contiguous and v_cache.flags.c_contiguous and k_cache.flags.writeable
+                and v_cache.flags.writeable):
+            raise ValueError("in-place write needs C-contiguous, writable caches")
+        kc, vc = k_cache, v_cache
+    else:
+        kc = np.array(k_cache, copy=True, order="C")
+        vc = np.array(v_cache, copy=True, order="C")
     sm = _c(slot_mapping, np.int64)
     NB, bs, Hk, D = kc.shape
     token_bytes = Hk * D * kc.itemsize

@@ -96,6 +96,10 @@ struct DecodeGeometry {
     int64_t ws_bytes;
 };
 
+int64_t round16(int64_t n) { return (n + 15) / 16 * 16; }
+
+// Workspace layout (split contexts only): fp32 O [B][H][P][D], then m and l
+// [B][H][P], then the fused merge's 64-bit tickets [B][Hk]; each 16-byte aligned.
 int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s,
                     DecodeGeometry *g) {
     if (num_seqs < 0 || max_context_len < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -107,8 +111,8 @@ int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested
         g->ws_bytes = 0;
     } else {
         const int64_t n = static_cast<int64_t>(num_seqs) * s->num_heads * g->max_parts;
-        const int64_t o_bytes = n * s->head_dim * 4;
-        g->ws_bytes = o_bytes + ((n * 4 + 15) / 16) * 16 * 2;
+        const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
+        g->ws_bytes = n * s->head_dim * 4 + round16(n * 4) * 2 + round16(units * 8);
     }
     return PA_OK;
 }
@@ -127,11 +131,45 @@ int allow_smem(K kernel, int bytes, std::atomic<uint64_t> &done) {
     return PA_OK;
 }
 
-constexpr int kStagePartitions = 1, kStageMerge = 2;
+// A stamp per launch for the fused merge's tickets: nonzero (a zeroed
+// workspace holds stamp 0) and different from the stamps of recent launches.
+// A launch captured in a CUDA graph keeps its stamp on every replay; its last
+// CTAs put the tickets back to (stamp, 0), so replays start afresh too.
+uint32_t next_stamp() {
+    static std::atomic<uint32_t> counter{0};
+    uint32_t s;
+    do {
+        s = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+    } while (s == 0);
+    return s;
+}
+
+// pa_decode: the split-context kernel with the merge fused into it.
+// pa_decode_partitions / pa_decode_merge: the split-context kernel without the
+// fused merge, and the merge as a kernel of its own.
+enum DecodeMode { kDecodeFused, kDecodePartitions, kDecodeMerge };
 
 template <typename Tq, typename Tc, int D, int G>
-int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, int stages) {
+int launch_decode(pa::DecodeParams prm, int num_seqs, cudaStream_t st, DecodeMode mode) {
     using C = pa::DecodeCfg<Tc, D, G>;
+    // Both kernels are programmatic dependent launches: each starts launching
+    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
+    // before reading anything.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (mode == kDecodeMerge) {
+        if (prm.max_parts == 1) return PA_OK;  // no context is split
+        cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
+        cfg.blockDim = dim3(G * D);
+        cfg.dynamicSmemBytes = 0;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
+        return e == cudaSuccess ? PA_OK : cuda_fail(e);
+    }
     static std::atomic<uint64_t> smem_done{0};
     int arc = allow_smem(pa::decode_kernel<Tq, Tc, D, G>, C::SMEM, smem_done);
     if (arc != PA_OK) return arc;
@@ -142,38 +180,22 @@ int launch_decode(const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, in
         !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
         return PA_ERR_UNSUPPORTED;
-    // Both kernels are programmatic dependent launches: each starts launching
-    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
-    // before reading anything.
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
+    prm.fuse_merge = mode == kDecodeFused ? 1 : 0;
+    prm.stamp = next_stamp();
     cfg.gridDim = dim3(prm.num_kv_heads, num_seqs, prm.max_parts);
     cfg.blockDim = dim3(pa::kDecodeThreads);
     cfg.dynamicSmemBytes = C::SMEM;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (stages & kStagePartitions) {
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
-    if (prm.max_parts == 1 || !(stages & kStageMerge)) return PA_OK;
-    cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
-    cfg.blockDim = dim3(G * D);
-    cfg.dynamicSmemBytes = 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
 template <typename Tq, typename Tc, int D>
-int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, int stages) {
+int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, DecodeMode mode) {
     switch (g) {
-        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st, stages);
-        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st, stages);
-        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st, stages);
-        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st, stages);
+        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st, mode);
+        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st, mode);
+        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st, mode);
+        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st, mode);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -248,7 +270,7 @@ namespace {
 int decode_stages(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                   int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
                   float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
-                  const pa_shape *shape, void *stream, int stages) {
+                  const pa_shape *shape, void *stream, DecodeMode mode) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -270,7 +292,8 @@ int decode_stages(void *out, const void *q, const void *k_cache, const void *v_c
         char *w = static_cast<char *>(workspace);
         prm.ws_o = reinterpret_cast<float *>(w);
         prm.ws_m = reinterpret_cast<float *>(w + n * shape->head_dim * 4);
-        prm.ws_l = reinterpret_cast<float *>(w + n * shape->head_dim * 4 + ((n * 4 + 15) / 16) * 16);
+        prm.ws_l = reinterpret_cast<float *>(w + n * shape->head_dim * 4 + round16(n * 4));
+        prm.ws_ticket = reinterpret_cast<unsigned long long *>(w + n * shape->head_dim * 4 + round16(n * 4) * 2);
     }
     prm.out = out;
     prm.q = q;
@@ -294,16 +317,16 @@ int decode_stages(void *out, const void *q, const void *k_cache, const void *v_c
     const int G = shape->num_heads / shape->num_kv_heads;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (shape->kv_fp8) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st, stages)
-                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st, stages);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st, mode)
+                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st, mode);
     }
     if (shape->dtype == PA_DTYPE_BF16) {
         return shape->head_dim == 128
-                   ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st, stages)
-                   : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st, stages);
+                   ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st, mode)
+                   : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st, mode);
     }
-    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st, stages)
-                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st, stages);
+    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st, mode)
+                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st, mode);
 }
 
 }  // namespace
@@ -316,7 +339,7 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               void *stream) {
     return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                          max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kStagePartitions | kStageMerge);
+                         kDecodeFused);
 }
 
 int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -325,7 +348,7 @@ int pa_decode_partitions(void *out, const void *q, const void *k_cache, const vo
                          void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream) {
     return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                          max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kStagePartitions);
+                         kDecodePartitions);
 }
 
 int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -334,7 +357,7 @@ int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v
                     int64_t workspace_bytes, const pa_shape *shape, void *stream) {
     return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                          max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kStageMerge);
+                         kDecodeMerge);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -370,18 +393,47 @@ namespace {
 // cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
-std::atomic<void *> g_noalloc_ptr[kMaxDevices];
+// Per device: the context the address was looked up in, and the address. A
+// context change (cudaDeviceReset, then a new primary context) reloads the
+// module, possibly elsewhere, so the address is looked up again.
+struct NoallocSlot {
+    std::atomic<void *> ctx{nullptr};
+    std::atomic<void *> ptr{nullptr};
+};
+NoallocSlot g_noalloc[kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+void *current_context() {
+    static CtxGetCurrentFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<CtxGetCurrentFn>(nullptr);
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return static_cast<void *>(c);
+}
 
 int noalloc_scratch(void **ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kMaxDevices) return PA_ERR_DEVICE;
-    void *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
+    NoallocSlot &slot = g_noalloc[dev];
+    void *ctx = current_context();
+    // ctx is stored after ptr and loaded before it: a matching ctx comes with its ptr
+    const void *seen_ctx = slot.ctx.load(std::memory_order_acquire);
+    void *p = slot.ptr.load(std::memory_order_acquire);
+    if (!p || !ctx || seen_ctx != ctx) {
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with `dev` current
         if (e != cudaSuccess) return cuda_fail(e);
-        g_noalloc_ptr[dev].store(p, std::memory_order_release);
+        if (!ctx) ctx = current_context();  // the lookup made the primary context current
+        slot.ptr.store(p, std::memory_order_release);
+        slot.ctx.store(ctx, std::memory_order_release);
     }
     *ptr = p;
     return PA_OK;
@@ -403,8 +455,13 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
         const int rc = noalloc_scratch(&scratch);
         if (rc != PA_OK) return rc;
     }
-    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                     max_context_len, scale, partition_tokens, scratch, need, shape, stream);
+    // The two-kernel form (split-context pass, then the merge kernel) keeps no
+    // state between calls in the scratch: nothing in it has to start at zero.
+    int rc = decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                           max_context_len, scale, partition_tokens, scratch, need, shape, stream, kDecodePartitions);
+    if (rc != PA_OK) return rc;
+    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                         max_context_len, scale, partition_tokens, scratch, need, shape, stream, kDecodeMerge);
 }
 
 static int launch_copy(void *dst, const void *src, const int64_t *pairs, int64_t num_pairs, int64_t src_blocks,

@@ -25,6 +25,8 @@ PA_STATUS_BAD_SLOT = 0x2
 PA_STATUS_BAD_CONTEXT = 0x4
 PA_STATUS_WAIT_TIMEOUT = 0x8
 PA_STATUS_BAD_QUERY = 0x10
+PA_STATUS_BAD_WORKSPACE = 0x20
+PA_ABI_VERSION = 4
 
 
 class PaShape(ctypes.Structure):
@@ -84,6 +86,9 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 lib = _load()
+if lib.pa_abi_version() != PA_ABI_VERSION:
+    raise ImportError("libpa.so has ABI version %d, the binding expects %d: rebuild it"
+                      % (lib.pa_abi_version(), PA_ABI_VERSION))
 
 
 class PaError(RuntimeError):
@@ -224,22 +229,23 @@ def pa_decode_merge(out, q, k_cache, v_cache, block_tables, context_lens, max_co
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
-                      partition_tokens: int = 0, stream=None) -> None:
+                      partition_tokens: int = 0, stream=None, k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """pa_decode without a workspace argument, for callers that cannot allocate device memory.
 
     The split-context partials go to a PA_NOALLOC_SCRATCH_BYTES array built
     into the library (held on every device that loads it). Requests that need
     more raise PaError with PA_ERR_SCRATCH_LIMIT. Calls that may overlap on
     one GPU share that array and must not run concurrently. Make the first
-    call on each device outside stream capture.
+    call on each device outside stream capture. A uint8 (FP8 E4M3) pool takes
+    k_scale and v_scale as in pa_decode.
     """
-    _same_dtype(out, q, k_cache, v_cache)
+    _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(context_lens, torch.int32, "context_lens")
     B, H, D = q.shape
     if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
-    shape = shape_of(k_cache, H)
+    shape = shape_of(k_cache, H, k_scale, v_scale)
     _check("pa_decode_noalloc",
            lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),

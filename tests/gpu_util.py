@@ -1,6 +1,8 @@
 """Helpers for the GPU parity tests: upload a PagedCase, run the library, compare with the oracle."""
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 import torch
 
@@ -59,3 +61,14 @@ def max_err(gpu_out: np.ndarray, ref: np.ndarray) -> float:
     if not np.all(np.isfinite(g)):
         return float("inf")
     return float(np.abs(g - ref).max()) if g.size else 0.0
+
+
+@functools.lru_cache(maxsize=1)
+def mixed_step_reference():
+    """The mixed step (a 2048-token chunk at offset 6144 and 192 decode tokens) with the oracle's
+    written caches and its attention for every one of the 2240 query rows, computed once per
+    test session."""
+    case = W.mixed_step()
+    kc, vc = oracle_written(case)
+    ref = oracle.prefill(case.q, kc, vc, case.block_tables, case.cu_q_lens, case.context_lens, case.scale)
+    return case, ref

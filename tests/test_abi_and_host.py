@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_messages():
     from paged_kv_cache_366_b200 import pa
-    assert pa.pa_abi_version() == 3
+    assert pa.pa_abi_version() == 4
     assert pa.pa_strerror(0) == "ok"
     assert "workspace" in pa.pa_strerror(-4)
     assert pa.pa_strerror(-99) == "unknown error"
@@ -52,16 +52,18 @@ def test_workspace_sizes():
     s = shape()
     # single pass for short contexts: no workspace
     assert pa.pa_decode_workspace_bytes(64, 300, 0, s) == 0
-    # split contexts: [B][H][P] m and l plus [B][H][P][D] partial outputs, fp32
+    # split contexts: [B][H][P] m and l plus [B][H][P][D] partial outputs, fp32, then the
+    # fused merge's 64-bit tickets [B][Hk]
     n = 64 * 32 * 4
-    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == n * 128 * 4 + 2 * ((n * 4 + 15) // 16 * 16)
+    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == (n * 128 * 4 + 2 * ((n * 4 + 15) // 16 * 16) +
+                                                             (64 * 8 * 8 + 15) // 16 * 16)
     with pytest.raises(pa.PaError):
         pa.pa_decode_workspace_bytes(4, 100, 100, s)  # not a multiple of 64
 
 
-def ws_bytes(B, H, P, D=128):
+def ws_bytes(B, H, P, D=128, Hk=8):
     n = B * H * P
-    return n * D * 4 + 2 * ((n * 4 + 15) // 16 * 16)
+    return n * D * 4 + 2 * ((n * 4 + 15) // 16 * 16) + (B * Hk * 8 + 15) // 16 * 16
 
 
 def test_automatic_partitions():

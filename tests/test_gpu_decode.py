@@ -195,3 +195,56 @@ def test_partitions_then_merge_equals_pa_decode(pa, name):
     torch.cuda.synchronize()
     assert pa.pa_get_status() == 0
     assert torch.equal(whole.view(torch.int16), parts.view(torch.int16))
+
+
+def test_workspace_needs_no_initialisation(pa):
+    # The fused merge's tickets carry a per-call stamp, so a workspace holding
+    # random bytes, or the leftovers of a call of another geometry, gives the
+    # same result as a fresh one.
+    big = W.make_case("ws_big", 31, context_lens=[4000, 2500, 900, 3333, 1500, 64], q_lens=[1] * 6, num_heads=32,
+                      num_kv_heads=8, head_dim=128, dtype="bf16")
+    small = W.make_case("ws_small", 32, context_lens=[1200, 700, 2049], q_lens=[1] * 3, num_heads=32,
+                        num_kv_heads=8, head_dim=128, dtype="bf16")
+    shape_b = pa.shape_of(to_dev(big.k_cache), 32)
+    n = max(pa.pa_decode_workspace_bytes(6, 4000, 128, shape_b), pa.pa_decode_workspace_bytes(3, 2049, 128, shape_b))
+    g = torch.Generator(device="cuda").manual_seed(5)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, device="cuda", generator=g)
+    for case in (big, small, big):  # the second and third calls start on the earlier calls' leftovers
+        d = DevCase(case)
+        pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+        out = torch.full_like(d.q, float("nan"))
+        mx = int(case.context_lens.max())
+        pa.pa_decode(out, d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, 128, ws)
+        assert pa.pa_get_status() == 0
+        kc_ref, vc_ref = oracle_written(case)
+        ref = oracle.decode(case.q, kc_ref, vc_ref, case.block_tables, case.context_lens, case.scale)
+        assert max_err(to_host(out), ref) <= TOL["bf16"], case.name
+
+
+def test_graph_replays_with_new_queries(pa):
+    # a captured pa_decode keeps its stamp; every replay must merge afresh
+    case = W.make_case("replay", 33, context_lens=[3000, 1000, 4096, 17], q_lens=[1] * 4, num_heads=32,
+                       num_kv_heads=8, head_dim=128, dtype="bf16")
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    shape = pa.shape_of(d.k_cache, 32)
+    ws = torch.zeros(pa.pa_decode_workspace_bytes(4, 4096, 256, shape), dtype=torch.uint8, device="cuda")
+    q = d.q.clone()
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        pa.pa_decode(out, q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, 4096, case.scale, 256, ws)
+    s.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=s):
+        pa.pa_decode(out, q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, 4096, case.scale, 256, ws)
+    kc_ref, vc_ref = oracle_written(case)
+    rng = np.random.default_rng(34)
+    for _ in range(3):
+        q_np = W.f32_to_bf16_bits(rng.uniform(-1, 1, case.q.shape).astype(np.float32))
+        q.copy_(to_dev(q_np))
+        gr.replay()
+        torch.cuda.synchronize()
+        ref = oracle.decode(q_np, kc_ref, vc_ref, case.block_tables, case.context_lens, case.scale)
+        assert max_err(to_host(out), ref) <= TOL["bf16"]
+    assert pa.pa_get_status() == 0

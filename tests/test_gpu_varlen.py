@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from paged_kv_cache_366_b200 import workloads as W
-from gpu_util import TOL, DevCase, max_err, oracle_written, to_host, widen
+from gpu_util import TOL, DevCase, max_err, mixed_step_reference, oracle_written, to_host, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -98,10 +98,8 @@ def test_spec_verify_full_size(pa):
 
 
 def test_mixed_step_in_one_launch_full_size(pa):
-    # the mixed step (2048-token chunk + 192 decode tokens) as one launch: all decode rows and
-    # sampled chunk rows, the chunk's first and last rows included
-    case = W.mixed_step()
-    rng = np.random.default_rng(65)
-    chunk = np.concatenate([[0, 1, 127, 128, 2047], rng.choice(2048, 40, replace=False)])
-    rows = np.unique(np.concatenate([chunk, np.arange(2048, 2240)]))
-    check(pa, case, rows=rows)
+    # the mixed step (2048-token chunk + 192 decode tokens) as one launch: every one of the 2240 rows
+    case, ref = mixed_step_reference()
+    got = one_launch(pa, case)
+    err = max_err(got, ref)
+    assert err <= TOL["bf16"], err
