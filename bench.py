@@ -438,7 +438,6 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
     max_ctx = int(case.context_lens[dec].max()) if len(dec) else 0
     ws_n = pa.pa_decode_workspace_bytes(len(dec), max_ctx, 0, shape) if len(dec) else 0
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
-    ws_split = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
 
     if len(pre):
         p0, p1 = int(pre[0]), int(pre[-1]) + 1
@@ -453,15 +452,10 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
     def do_write():
         pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, k_scale=ks, v_scale=vs)
 
-    def do_decode():  # one kernel: the split-context pass with the merge fused in
+    def do_decode():  # one kernel: equal slices of the block list, cut units merged inside
         pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws,
                      k_scale=ks, v_scale=vs)
 
-    out_split = torch.empty_like(q_dec) if len(dec) else None
-
-    def do_partitions():  # the split-context pass alone, without the merge (not part of the step)
-        pa.pa_decode_partitions(out_split, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx,
-                                case.scale, 0, ws_split, k_scale=ks, v_scale=vs)
 
     def do_prefill():
         pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
@@ -483,8 +477,6 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
             parts.append(("prefill", do_prefill))
         if len(dec):
             parts.append(("decode", do_decode))
-            if ws_n:
-                extra.append(("partitions_only", do_partitions))
     launches_per_step = len(parts)
 
     # one graph for the whole step (the headline), one per part (breakdown, roofline)
@@ -601,12 +593,10 @@ def decode_roofline(m, peak, peak_kind, name):
     achieved = nb / t_dec / 1e9
     r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
          "frac_of_nominal": achieved / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
-         "traffic": profiled_traffic(name), "kernel": "decode_kernel (split-context pass with the merge fused in; "
-                                                      "the whole pa_decode call)",
+         "traffic": profiled_traffic(name), "kernel": "decode_kernel (the whole pa_decode call: one launch, "
+                                                      "equal slices per CTA, cut units merged inside)",
          "algorithmic_bytes_per_launch": nb, "us_per_launch": t_dec * 1e6,
          "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind}
-    if "partitions_only" in m["per_part"]:
-        r["partition_pass_alone_us"] = m["per_part"]["partitions_only"] * 1e6
     return r
 
 

@@ -79,7 +79,6 @@ typedef enum {
 #define PA_STATUS_BAD_CONTEXT 0x4u    /* context length < 0, > MB * 16, or > max_context_len */
 #define PA_STATUS_WAIT_TIMEOUT 0x8u   /* a bounded wait on an async copy gave up */
 #define PA_STATUS_BAD_QUERY 0x10u     /* prefill: q_len > context_len or cu_q_lens not increasing */
-#define PA_STATUS_BAD_WORKSPACE 0x20u /* pa_decode: a merge ticket had more arrivals than partitions */
 
 typedef struct {
     int32_t num_heads;    /* H, query heads */
@@ -129,11 +128,12 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
 
 /*
  * pa_decode_workspace_bytes: scratch size pa_decode needs for these sizes
- * and this partition_tokens (0 = automatic), on the current device. It is 0
- * when no context is split across partitions. Negative on bad arguments.
- * Layout: fp32 partial outputs [B][H][P][D], partial maxima and sums
- * [B][H][P] each, then 64-bit merge tickets [B][Hk], each part 16-byte
- * aligned.
+ * and this partition_tokens (0 = automatic), on the current device; 0 only
+ * when num_seqs is 0. Negative on bad arguments.
+ * With S slices (see pa_decode) and U = B * Hk units the layout is: fp32
+ * partial outputs [S + U - 1][G][D], partial maxima and sums [S + U - 1][G]
+ * each, then int32 (first slice, slices) records [U], each part 16-byte
+ * aligned (G = H / Hk).
  */
 int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int32_t partition_tokens,
                                   const pa_shape *shape);
@@ -156,51 +156,29 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
  *                  it sizes the grid and the workspace. A device length above
  *                  it is clamped and sets PA_STATUS_BAD_CONTEXT.
  *   scale        : softmax scale (the sketch has none; typically 1/sqrt(D))
- *   partition_tokens : 0 = automatic. Otherwise tokens per split-context
- *                  partition, a multiple of 64 and >= 64. A context longer
- *                  than one partition is split. Each partition writes
- *                  (max, sum, unnormalised O) to the workspace; the last
- *                  partition of a (sequence, KV head) to finish, found by a
- *                  ticket counter in the workspace, merges them. pa_decode is
- *                  one kernel launch.
+ *   partition_tokens : 0 = automatic. The list of (sequence, KV head,
+ *                  16-token block) items is cut into S equal slices, one per
+ *                  warp of a persistent grid; a (sequence, KV head) cut by
+ *                  slice boundaries gets one partial (max, sum, unnormalised
+ *                  O) per slice in the workspace, and a second kernel merges
+ *                  them. Automatic S: the warps of all the decode CTAs the SMs
+ *                  hold at once, at most one per 4 blocks of
+ *                  B * Hk * ceil(max_context_len / 16). Otherwise a multiple
+ *                  of 64, >= 64: S makes a slice about partition_tokens tokens
+ *                  of a context of max_context_len (a smaller value means
+ *                  more, smaller slices).
  *   workspace    : device scratch of >= pa_decode_workspace_bytes(...) bytes,
- *                  16-byte aligned. It may be NULL when that size is 0. Its
- *                  contents need no initialisation: each merge ticket holds a
- *                  stamp of the call that wrote it (different for every host
- *                  call, kept by a CUDA graph replay, which leaves its tickets
- *                  reset), and a ticket with another stamp counts as empty. A
- *                  ticket with this call's stamp and too many arrivals (two
- *                  overlapping replays of one graph, say) sets
- *                  PA_STATUS_BAD_WORKSPACE. Calls that overlap on the GPU must
- *                  not share a workspace.
+ *                  16-byte aligned. Its contents need no initialisation: a
+ *                  call writes every partial and record before it reads it.
+ *                  Calls that overlap on the GPU must not share a workspace.
  * Accumulation is fp32 whatever the dtype. bf16 output is rounded once, to
- * nearest even.
+ * nearest even. Two kernel launches, the second a programmatic dependent of
+ * the first.
  */
 int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
               int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
               float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
               const pa_shape *shape, void *stream);
-
-/*
- * pa_decode_partitions, pa_decode_merge: pa_decode as two kernels, one call
- * each. They take exactly pa_decode's arguments, and pa_decode_partitions
- * followed by pa_decode_merge on the same stream with the same arguments gives
- * pa_decode's result bit for bit. pa_decode_partitions runs the split-context
- * pass without the fused merge: sequences of one partition write out
- * directly, longer ones write their partials to the workspace.
- * pa_decode_merge combines those partials into out; it does nothing when no
- * context is split. Neither touches the merge tickets, so the workspace needs
- * no zeroing for them. Exposed so a caller can put other work between the two
- * or time each kernel. Errors as for pa_decode.
- */
-int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
-                         const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
-                         int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
-                         void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream);
-int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
-                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
-                    int64_t workspace_bytes, const pa_shape *shape, void *stream);
 
 /*
  * pa_prefill_chunk: causal attention for chunks of query tokens placed at a
@@ -293,11 +271,9 @@ int pa_swap_blocks(void *dst, const void *src, const int64_t *block_pairs, int64
  *    partition_tokens.
  *  - Every call on a device shares the one array, and the array keeps whatever
  *    the last call left in it. Nothing in it needs to start at zero: a call
- *    runs pa_decode as its two kernels (pa_decode_partitions, then
- *    pa_decode_merge), and the first writes every partial the second reads.
- *    Calls that may overlap on the GPU (different streams, or different host
- *    threads on one device) race on the array and must be serialized by the
- *    caller.
+ *    writes every partial and record before it reads it. Calls that may
+ *    overlap on the GPU (different streams, or different host threads on one
+ *    device) race on the array and must be serialized by the caller.
  * The library calls no cudaMalloc, cudaFree or other allocating routine here.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -8,20 +8,26 @@
 // a running result. That is online softmax: a running max m, a running sum l
 // and an accumulator O rescaled by exp(m_old - m_new) whenever m grows.
 //
-// How it runs on B200:
-//  * Grid (KV head, sequence, partition). A CTA owns one KV head of one
-//    sequence over one partition of the context (split-context pass).
-//    Sequences longer than a partition write (m, l, O) partials, and the last
-//    CTA of the (sequence, KV head) to finish merges them (a ticket counter in
-//    the workspace), so pa_decode is one kernel. The merge can also run as its
-//    own kernel (decode_reduce_kernel), with the same arithmetic.
+// How it runs on B200 (two kernels, the second a programmatic dependent):
+//  * Work is the flat list of (sequence, KV head, block) triples in that
+//    order; a (sequence, KV head) pair is a "unit". The grid is persistent
+//    (the CTAs all SMs hold at once) and each warp takes one of
+//    4 * gridDim.x equal, contiguous slices of the list, so every warp gets
+//    the same number of blocks (to one) whatever the mix of lengths: no tail
+//    of short CTAs, no empty CTAs, one prologue per CTA. A CTA finds its
+//    warps' slices by a prefix sum of the sequences' block counts, read from
+//    context_lens on the device. After that the warps run independently.
+//  * A unit's part inside one slice is a "segment". A warp leaving a segment
+//    writes the unit's output itself when the whole unit lies in its slice;
+//    otherwise it writes the segment's partial (m, l, O) to the workspace.
+//    decode_merge_kernel then merges the partials of every cut unit.
 //  * Every query head of the KV head's group (G = H / Hk of them) reads each
 //    loaded block from shared memory, so K/V cross HBM once per KV head.
-//  * The 4 warps of a CTA take the partition's blocks round-robin. Each warp
-//    streams its own blocks through an NSTAGE-deep shared-memory ring. A
-//    block's 16 K rows and 16 V rows of one KV head are two TMA tiled loads
+//  * Each warp streams its blocks through an NSTAGE-deep shared-memory ring:
+//    a block's 16 K rows and 16 V rows of one KV head are two TMA tiled loads
 //    (a [16][D] box of the pool viewed as [NB*16][Hk][D]) into a ring slot,
-//    and an mbarrier counts the bytes. Fetches run NSTAGE blocks ahead.
+//    and an mbarrier counts the bytes. Fetches run NSTAGE blocks ahead,
+//    across segment boundaries.
 //  * Lanes own column slices of a row made of CH chunks of CB bytes,
 //    interleaved so shared-memory reads are conflict free. L lanes cover a
 //    row and RS = 32 / L rows are processed per step.
@@ -38,8 +44,6 @@
 //    lane exponentiates its own scores and stores them, duplicated as packed
 //    pairs, in a small per-warp buffer that P.V reads back as broadcasts.
 //  * P.V uses packed two-wide fp32 FMAs on (even, odd) column pairs.
-//  * Each warp keeps its own (m, l, O). At the end the warps merge through
-//    shared memory (reusing the ring).
 #pragma once
 
 #include <math_constants.h>
@@ -56,10 +60,12 @@ template <typename T, int D, int G>
 struct DecodeCfg {
     static constexpr int E = sizeof(T);
     static constexpr int R = D * E;                        // bytes of one token row of one KV head
-    // Bytes of one chunk: 16, or 8 for FP8 rows with groups of 8 heads, so that
-    // a lane holds 8 dims per row as for bf16 (16 would spill q and O).
-    static constexpr int CB = (E == 1 && G >= 8) ? 8 : 16;
-    static constexpr int CH = (G >= 8 || E == 1) ? 1 : 2;  // chunks a lane owns per row
+    // Bytes of one chunk: 16, or 8 for FP8 rows, so that a lane holds 8 dims
+    // per chunk as for bf16 (16 would spill q and O).
+    static constexpr int CB = E == 1 ? 8 : 16;
+    // One chunk per lane and row: q and O then take 64 registers for 4 heads
+    // (two chunks spill at three CTAs per SM).
+    static constexpr int CH = 1;
     static constexpr int L = R / (CB * CH);                // lanes covering one row
     static constexpr int RS = 32 / L;                      // rows per warp step
     static constexpr int STEPS = kBlockSize / RS;          // steps per block
@@ -69,40 +75,30 @@ struct DecodeCfg {
     static constexpr int STAGE_BYTES = 2 * kBlockSize * R; // K and V of one block
     // Two stages per warp and three CTAs per SM (12 warps) measured faster on
     // B200 than three stages at two CTAs per SM.
-#ifndef PA_DECODE_NSTAGE
-#define PA_DECODE_NSTAGE 2
-#endif
-#ifndef PA_DECODE_PF
-#define PA_DECODE_PF 0
-#endif
-    static constexpr int NSTAGE = PA_DECODE_NSTAGE;
-    // Blocks ahead of the one being loaded into shared memory whose K and V
-    // are prefetched into L2 (0: none).
-    static constexpr int PF = PA_DECODE_PF;
+    static constexpr int NSTAGE = 2;
     // CTAs per SM the register budget is sized for (wide rows keep more live state).
-#ifndef PA_DECODE_MINB4
-#define PA_DECODE_MINB4 3
-#endif
-    static constexpr int MIN_BLOCKS = G <= 4 ? PA_DECODE_MINB4 : 2;
+    static constexpr int MIN_BLOCKS = G <= 4 ? 3 : 2;
     static constexpr int WARP_RING = NSTAGE * STAGE_BYTES;
     static constexpr int RING_BYTES = kDecodeWarps * WARP_RING;
     static constexpr int NPART = STEPS * G;                 // q.k partials per lane per block
     static constexpr int NFIN = NPART >= L ? NPART / L : 1; // complete scores per lane
     static constexpr int DUP = NPART >= L ? 1 : L / NPART;  // lanes holding the same scores
     static constexpr int PBUF = kBlockSize * G * 8;         // per warp: [16 rows][G heads] of (p, p)
-    static constexpr int RED_BYTES = kDecodeWarps * RS * G * D * 4;
-    static constexpr int BIG = RING_BYTES > RED_BYTES ? RING_BYTES : RED_BYTES;
-    static constexpr int OFF_BAR = BIG;
+    static constexpr int OFF_BAR = RING_BYTES;              // NSTAGE mbarriers per warp
     static constexpr int OFF_P = OFF_BAR + kDecodeWarps * NSTAGE * 8;
-    static constexpr int OFF_ML = OFF_P + kDecodeWarps * PBUF;
-    static constexpr int OFF_FLAG = OFF_ML + 2 * kDecodeWarps * G * 4;
-    static constexpr int SMEM = OFF_FLAG + 16;
+    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;  // the warps' slice starts
+    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16;
+    // CTAs of this kernel one SM holds: the register budget or shared memory
+    // (228 KB per SM, 1 KB of it reserved per CTA), whichever binds first.
+    static constexpr int RESIDENT = (228 * 1024) / (SMEM + 1024) < MIN_BLOCKS ? (228 * 1024) / (SMEM + 1024)
+                                                                              : MIN_BLOCKS;
     static_assert(R % (CB * CH) == 0 && L >= 1 && L <= 32 && 32 % L == 0, "row must split into lane slices");
     static_assert(kBlockSize % RS == 0, "rows per step must divide the block");
     static_assert(32 % G == 0 && G <= 8, "group size");
     static_assert(G % NFIN == 0, "a lane's scores are consecutive heads of one row");
-    static_assert(OFF_P % 16 == 0, "probability buffer alignment");
+    static_assert(OFF_P % 16 == 0 && OFF_MISC % 16 == 0, "shared-memory alignment");
     static_assert(STEPS >= 2 && L >= 4, "the first reduce step pairs step slots s and s + STEPS / 2");
+    static_assert(RESIDENT >= 1, "one CTA must fit an SM");
 };
 
 // Sum, over the lanes that differ in the bits OFF, OFF/2, ..., 1, the N values
@@ -161,114 +157,61 @@ struct DecodeParams {
     const void *v_cache;
     const int *block_tables;
     const int *context_lens;
-    float *ws_o;  // [B][H][max_parts][D]
-    float *ws_m;  // [B][H][max_parts]
-    float *ws_l;  // [B][H][max_parts]
-    unsigned long long *ws_ticket;  // [B][Hk] tickets of the fused merge: (call stamp << 32) | arrivals
+    float *ws_o;   // [slots][G][D] partial outputs; slot = slice index + unit index
+    float *ws_m;   // [slots][G]
+    float *ws_l;   // [slots][G]
+    int *ws_unit;  // [B][Hk][2]: (first slice, slices) of each unit with blocks, written every call
     long long num_blocks;
+    int num_seqs;
     int max_blocks_per_seq;
     int num_heads;
     int num_kv_heads;
     int max_context_len;
-    int part_tokens;
-    int max_parts;
-    int fuse_merge;    // 1: the last partition CTA of a unit merges; 0: decode_reduce_kernel does
-    unsigned int stamp;  // nonzero, different for every host call: a ticket with another stamp counts as 0
     float scale_log2;  // softmax scale * log2(e) (times k_scale for an FP8 cache)
     float v_scale;     // 1, or the FP8 value scale
 };
 
-// Merge the `parts` partials of query head h of sequence b for column d:
-//   M = max_p m_p,  L = sum_p 2^(m_p - M) l_p,  out = sum_p 2^(m_p - M) O_p / L,
-// in one pass with a running max, loading up to 8 partitions at a time.
-// The fused merge and decode_reduce_kernel share it, so both give the same bits.
-template <typename T>
-__device__ __forceinline__ void merge_partitions(const DecodeParams &prm, int b, int h, int parts, int d, int D) {
-    const size_t base = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts;
-    float M = -CUDART_INF_F, O = 0.f, L = 0.f;
-    for (int p0 = 0; p0 < parts; p0 += 8) {
-        float mp[8], lp[8], op[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const bool in = p0 + i < parts;
-            mp[i] = in ? __ldcg(prm.ws_m + base + p0 + i) : -CUDART_INF_F;
-            lp[i] = in ? __ldcg(prm.ws_l + base + p0 + i) : 0.f;
-            op[i] = in ? __ldcg(prm.ws_o + (base + p0 + i) * D + d) : 0.f;
-        }
-        float mc = M;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
-        if (mc == -CUDART_INF_F) continue;
-        const float a = exp2f(M - mc);  // 0 while M is still -inf
-        O *= a;
-        L *= a;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float wt = mp[i] == -CUDART_INF_F ? 0.f : exp2f(mp[i] - mc);
-            O += wt * op[i];
-            L += wt * lp[i];
-        }
-        M = mc;
-    }
-    T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
-    store_out(out, L > 0.f ? O / L : 0.f);
+// Position in the flat (sequence, KV head, block) list.
+struct Cursor {
+    int r;      // flat index minus the slice's first index
+    int b, hk;  // the unit
+    int c;      // context length of b (clamped)
+    int nblk;   // blocks of the unit
+    int blk;    // block within the unit
+};
+
+__device__ __forceinline__ int decode_cap(const DecodeParams &prm) {
+    return min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
 }
 
-// merge_partitions for up to NE output elements of one (sequence, KV head)
-// group at once, elements idx0 + e * stride (e < NE, below `total`) of its
-// [G][D] outputs, with the loads of all of them in flight together. Per
-// element, the arithmetic is merge_partitions' (the same bits).
-template <typename T, int NE>
-__device__ __forceinline__ void merge_partitions_n(const DecodeParams &prm, int b, int h0, int idx0, int stride,
-                                                   int total, int parts, int D) {
-    size_t base[NE];
-    int dd[NE];
-    float M[NE], O[NE], L[NE];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-        const int idx = min(idx0 + e * stride, total - 1);  // past the end: a copy of the last, not stored
-        base[e] = (static_cast<size_t>(b) * prm.num_heads + h0 + idx / D) * prm.max_parts;
-        dd[e] = idx % D;
-        M[e] = -CUDART_INF_F;
-        O[e] = 0.f;
-        L[e] = 0.f;
-    }
-    for (int p0 = 0; p0 < parts; p0 += 8) {
-        float mp[NE][8], lp[NE][8], op[NE][8];
-#pragma unroll
-        for (int e = 0; e < NE; ++e)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const bool in = p0 + i < parts;
-                mp[e][i] = in ? __ldcg(prm.ws_m + base[e] + p0 + i) : -CUDART_INF_F;
-                lp[e][i] = in ? __ldcg(prm.ws_l + base[e] + p0 + i) : 0.f;
-                op[e][i] = in ? __ldcg(prm.ws_o + (base[e] + p0 + i) * D + dd[e]) : 0.f;
-            }
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
-            float mc = M[e];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[e][i]);
-            if (mc == -CUDART_INF_F) continue;
-            const float a = exp2f(M[e] - mc);  // 0 while M is still -inf
-            O[e] *= a;
-            L[e] *= a;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float wt = mp[e][i] == -CUDART_INF_F ? 0.f : exp2f(mp[e][i] - mc);
-                O[e] += wt * op[e][i];
-                L[e] += wt * lp[e][i];
-            }
-            M[e] = mc;
+// Move x forward by n positions; returns the number of units left behind.
+// Sequences of length 0 hold no blocks and are stepped over.
+__device__ __forceinline__ int cursor_advance(Cursor &x, int n, const DecodeParams &prm) {
+    x.r += n;
+    x.blk += n;
+    int passed = 0;
+    while (x.blk >= x.nblk) {
+        x.blk -= x.nblk;
+        ++passed;
+        if (++x.hk == prm.num_kv_heads) {
+            x.hk = 0;
+            do {
+                if (++x.b >= prm.num_seqs) {  // past the end of the list: never used for a block
+                    x.nblk = 1 << 30;
+                    return passed;
+                }
+                x.c = clamp_context(__ldg(prm.context_lens + x.b), decode_cap(prm), false);
+            } while (x.c == 0);
+            x.nblk = (x.c + kBlockSize - 1) / kBlockSize;
         }
     }
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-        const int idx = idx0 + e * stride;
-        if (idx >= total) break;
-        T *out = static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h0 + idx / D) * D + dd[e];
-        store_out(out, L[e] > 0.f ? O[e] / L[e] : 0.f);
-    }
+    return passed;
+}
+
+// Slice holding flat index f when N items are cut into W slices
+// [s * N / W, (s + 1) * N / W).
+__device__ __forceinline__ int slice_of(long long f, long long N, int W) {
+    return static_cast<int>(((f + 1) * W - 1) / N);
 }
 
 // Tq: element type of q and out. Tc: element type of the caches (the same, or
@@ -280,12 +223,13 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     using C = DecodeCfg<Tc, D, G>;
     constexpr int P2 = C::P2;      // packed pairs per lane per row
     constexpr int VP = C::VE / 2;  // packed pairs per chunk
-    // Grid (KV head, sequence, partition): every unit's first partition launches
-    // before any second one, so full partitions run first and the short last
-    // partitions (or empty CTAs) form the tail.
-    const int hk = blockIdx.x, b = blockIdx.y, p = blockIdx.z;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int rg = lane / C::L, j = lane % C::L;
+    const int B = prm.num_seqs, Hk = prm.num_kv_heads;
+    const int cap = decode_cap(prm);
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    int *starts = reinterpret_cast<int *>(smem + C::OFF_MISC);  // per warp: b, hk, blk, c, nblk of its first block
 
     // The lane's step and head order for the transpose-reduce: at the reduce
     // step whose partner differs in lane bit `off`, values i and i + h (h half
@@ -310,52 +254,135 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     }
 
     // Launched as a programmatic dependent (its launch overlaps the previous
-    // kernel, e.g. the cache write): wait for that kernel before reading any input.
+    // kernel, e.g. the cache write): wait for that kernel before reading any
+    // input. The merge kernel that follows may start its launch at once; it
+    // waits for this grid to finish before reading anything.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int part_blocks = prm.part_tokens / kBlockSize;
-    const int blk0 = p * part_blocks;
-    const int *trow = prm.block_tables + static_cast<size_t>(b) * prm.max_blocks_per_seq + blk0;
-    // The length and this warp's first table entries load together (the
-    // entries are only used for blocks inside the context).
-    const int c_raw = __ldg(prm.context_lens + b);
-    const int tbl_lim = min(part_blocks, prm.max_blocks_per_seq - blk0);
-    int tbl = 0;
-    if (warp + lane * kDecodeWarps < tbl_lim) tbl = __ldg(trow + warp + lane * kDecodeWarps);
 
-    const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
-    const int c = clamp_context(c_raw, cap, p == 0 && hk == 0 && threadIdx.x == 0);
-    const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
-    if (p >= parts) return;
+    // ---- prologue (the whole CTA): the total block count N, the slices, and
+    // the unit holding each warp's first block
+    long long N = 0;
+    {
+        long long part = 0;
+        for (int b = threadIdx.x; b < B; b += kDecodeThreads) {
+            const int c = clamp_context(__ldg(prm.context_lens + b), cap, blockIdx.x == 0);
+            part += (c + kBlockSize - 1) / kBlockSize;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        long long *red64 = reinterpret_cast<long long *>(smem);
+        if (lane == 0) red64[warp] = part;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) N += red64[w];
+        N *= Hk;
+        __syncthreads();
+    }
+    // Sequences of length 0 have no blocks: CTA b % gridDim.x writes their zero rows.
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        if (clamp_context(__ldg(prm.context_lens + b), cap, false) != 0) continue;
+        Tq *o = static_cast<Tq *>(prm.out) + static_cast<size_t>(b) * prm.num_heads * D;
+        for (int i = threadIdx.x; i < prm.num_heads * D; i += kDecodeThreads) store_out(o + i, 0.f);
+    }
+    // WS slices, at most one per block, so that none is empty (a unit's slices
+    // are then exactly those from the slice of its first block to that of its last)
+    const int WS = static_cast<int>(min(static_cast<long long>(gridDim.x) * kDecodeWarps, N));
+    const int cta0 = static_cast<int>(blockIdx.x) * kDecodeWarps;  // first slice of this CTA
+    if (cta0 >= WS) return;
+    {
+        // Locate each warp's first block: prefix sums of Hk * blocks over the
+        // sequences, a chunk of sequences at a time in shared memory (the ring
+        // is not in use yet).
+        constexpr int CHUNK = C::RING_BYTES / 8;
+        long long *cum = reinterpret_cast<long long *>(smem);
+        long long base = 0;
+        for (int c0 = 0; c0 < B; c0 += CHUNK) {
+            const int n = min(CHUNK, B - c0);
+            for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
+                const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
+                cum[i] = static_cast<long long>((c + kBlockSize - 1) / kBlockSize) * Hk;
+            }
+            __syncthreads();
+            if (warp == 0) {  // inclusive scan, 32 entries per step
+                long long carry = base;
+                for (int i0 = 0; i0 < n; i0 += 32) {
+                    long long v = i0 + lane < n ? cum[i0 + lane] : 0;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const long long t = __shfl_up_sync(0xffffffffu, v, off);
+                        if (lane >= off) v += t;
+                    }
+                    v += carry;
+                    if (i0 + lane < n) cum[i0 + lane] = v;
+                    carry = __shfl_sync(0xffffffffu, v, 31);
+                }
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
+                const long long hi = cum[i], lo = i ? cum[i - 1] : base;
+                if (lo >= hi) continue;
+#pragma unroll
+                for (int w = 0; w < kDecodeWarps; ++w) {
+                    const long long f = N * (cta0 + w) / WS;  // first block of slice cta0 + w
+                    if (cta0 + w < WS && lo <= f && f < hi) {  // ... lies in sequence c0 + i
+                        const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
+                        const int nblk = (c + kBlockSize - 1) / kBlockSize;
+                        const long long r = f - lo;
+                        starts[5 * w + 0] = c0 + i;
+                        starts[5 * w + 1] = static_cast<int>(r / nblk);
+                        starts[5 * w + 2] = static_cast<int>(r % nblk);
+                        starts[5 * w + 3] = c;
+                        starts[5 * w + 4] = nblk;
+                    }
+                }
+            }
+            base = cum[n - 1];
+            __syncthreads();
+        }
+    }
+    // ---- from here on every warp runs alone on its slice
+    const int slice = cta0 + warp;
+    if (slice >= WS) return;
+    const long long s_lo = N * slice / WS, s_hi = N * (slice + 1) / WS;
+    const int nb_w = static_cast<int>(s_hi - s_lo);
 
-    const int nblk_seq = (c + kBlockSize - 1) / kBlockSize;
-    const int nb_cta = max(0, min(nblk_seq - blk0, part_blocks));
-    const int last_valid = c - (nblk_seq - 1) * kBlockSize;
-
-    extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *ring = smem + warp * C::WARP_RING;
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bars = smem_addr(smem + C::OFF_BAR) + warp * C::NSTAGE * 8;
     float *pbuf = reinterpret_cast<float *>(smem + C::OFF_P + warp * C::PBUF);  // [16][G] of (p, p)
     const uint32_t pbuf_s = smem_addr(pbuf);
-
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < C::NSTAGE; ++s) mbar_init(bars + 8 * s, 1);
         fence_mbar_init();
     }
     __syncwarp();
+    Cursor cc{0, starts[5 * warp], starts[5 * warp + 1], starts[5 * warp + 3], starts[5 * warp + 4],
+              starts[5 * warp + 2]};
 
-    // This warp's blocks: partition block warp + k * kDecodeWarps, k < nb_w.
-    const int nb_w = nb_cta > warp ? (nb_cta - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    // ---- issue side: block k of this warp at cursor ic (NSTAGE blocks ahead of
+    // the block being consumed), with the next 32 table entries of its unit
+    // (lane i holds block tbase + i)
+    int tb_u = -1, tbase = 0, tw = 0;
     uint32_t bad_mask = 0;
-
-    auto issue = [&](int k) {
-        if (k >= 32 && (k & 31) == 0) {
-            const int li = warp + (k + lane) * kDecodeWarps;
-            tbl = k + lane < nb_w && li < tbl_lim ? __ldg(trow + li) : 0;
+    auto issue = [&](int k, const Cursor &ic) {
+        const int u = ic.b * Hk + ic.hk;
+        if (u != tb_u || ic.blk >= tbase + 32) {
+            if (u != tb_u) {  // a new unit: bring its queries towards the SM while its blocks load
+                const char *qrow = static_cast<const char *>(prm.q) +
+                                   (static_cast<size_t>(ic.b) * prm.num_heads + ic.hk * G) * D * sizeof(Tq);
+                if (lane * 128 < G * D * static_cast<int>(sizeof(Tq)))
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + lane * 128));
+            }
+            tb_u = u;
+            tbase = ic.blk;
+            const int e = tbase + lane;
+            tw = e < min(ic.nblk, prm.max_blocks_per_seq)
+                     ? __ldg(prm.block_tables + static_cast<size_t>(ic.b) * prm.max_blocks_per_seq + e)
+                     : 0;
         }
-        int pb = __shfl_sync(0xffffffffu, tbl, k & 31);
+        int pb = __shfl_sync(0xffffffffu, tw, ic.blk - tbase);
         const int s = k % C::NSTAGE;
         if (pb < 0 || pb >= prm.num_blocks) {
             if (lane == 0) flag_status(PA_STATUS_BAD_BLOCK_ID);
@@ -368,32 +395,22 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         if (lane == 0) {
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
             const uint32_t dst = ring_s + s * C::STAGE_BYTES;
-            tma_load_3d(dst, &tm_k, 0, hk, pb * kBlockSize, bar);
-            tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, hk, pb * kBlockSize, bar);
+            tma_load_3d(dst, &tm_k, 0, ic.hk, pb * kBlockSize, bar);
+            tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar);
         }
     };
-    // L2 prefetch of block kp when it is inside the 32-entry table window of
-    // block kw, the block issued last.
-    auto prefetch = [&](int kp, int kw) {
-        if (C::PF == 0 || kp >= nb_w || (kp >> 5) != (kw >> 5)) return;
-        const int pb = __shfl_sync(0xffffffffu, tbl, kp & 31);
-        if (lane == 0 && pb >= 0 && pb < prm.num_blocks) {
-            tma_prefetch_l2_3d(&tm_k, 0, hk, pb * kBlockSize);
-            tma_prefetch_l2_3d(&tm_v, 0, hk, pb * kBlockSize);
+    {
+        Cursor ic = cc;
+        for (int i = 0; i < min(C::NSTAGE, nb_w); ++i) {
+            if (i) cursor_advance(ic, 1, prm);
+            issue(i, ic);
         }
-    };
-
-    int issued = 0;
-    for (; issued < min(C::NSTAGE, nb_w); ++issued) issue(issued);
-    if (C::PF > 0) {
-#pragma unroll 1
-        for (int kp = C::NSTAGE; kp < C::NSTAGE + C::PF; ++kp) prefetch(kp, 0);
     }
 
-    // Queries of the group in this lane's head order, pre-scaled by
+    // Queries of a unit in this lane's head order, pre-scaled by
     // scale * log2(e), as packed pairs of the lane's columns.
     f32x2 q2[G][P2];
-    {
+    auto load_q = [&](int b, int hk) {
         constexpr int QV = C::VE * static_cast<int>(sizeof(Tq)) / 16;  // 16-byte q loads per chunk
         constexpr int QP = Widen<Tq>::N / 2;                            // pairs per q load
         const Tq *qb = static_cast<const Tq *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
@@ -412,310 +429,335 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
                 for (int e = 0; e < VP; ++e) mul2(q2[g][ch * VP + e], sc);
             }
         }
-    }
+    };
 
     f32x2 acc2[G][P2];
+    float m_col;           // running max (log2 domain) of head lane % G
+    float l_f[C::NFIN];    // this lane's share of the running sums of heads hmask + f
+    float mu_f[C::NFIN];   // exponent reference of head hmask + f: its max, or 0 while -inf
+    float thr_f[C::NFIN];  // a score above this moves the max of head hmask + f
+    auto reset_state = [&]() {
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < P2; ++e) acc2[g][e] = 0ull;
-    float m_col = -CUDART_INF_F;  // running max (log2 domain) of head lane % G
-    float l_f[C::NFIN];           // this lane's share of the running sums of heads hmask + f
-    float mu_f[C::NFIN];          // exponent reference of head hmask + f: its max, or 0 while -inf
-    float thr_f[C::NFIN];         // a score above this moves the max of head hmask + f
+            for (int e = 0; e < P2; ++e) acc2[g][e] = 0ull;
+        m_col = -CUDART_INF_F;
 #pragma unroll
-    for (int f = 0; f < C::NFIN; ++f) {
-        l_f[f] = 0.f;
-        mu_f[f] = 0.f;
-        thr_f[f] = -CUDART_INF_F;
-    }
+        for (int f = 0; f < C::NFIN; ++f) {
+            l_f[f] = 0.f;
+            mu_f[f] = 0.f;
+            thr_f[f] = -CUDART_INF_F;
+        }
+    };
     const int t_own = smask * C::RS + rg;  // the row of this lane's scores
     const uint32_t p_own = pbuf_s + (t_own * G + hmask) * 8;
 
-    int k = 0;
-    bool failed = false;
-    for (; k < nb_w; ++k) {
-        const int s = k % C::NSTAGE;
-        const bool landed = mbar_wait(bars + 8 * s, (k / C::NSTAGE) & 1);
-        if (!__all_sync(0xffffffffu, landed)) {
-            failed = true;
-            break;
+    // ---- leave the segment of the unit at cc: the unit's output if the whole
+    // unit lies in this slice, else the segment's partial (m, l, O)
+    auto close_segment = [&]() {
+        // sum O over the row groups of the warp (lanes that differ in the row-group bits)
+#pragma unroll
+        for (int off = C::L; off < 32; off <<= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < P2; ++e) {
+                    float lo, hi;
+                    unpack2(acc2[g][e], lo, hi);
+                    lo += __shfl_xor_sync(0xffffffffu, lo, off);
+                    hi += __shfl_xor_sync(0xffffffffu, hi, off);
+                    acc2[g][e] = pack2(lo, hi);
+                }
+        if (C::DUP > 1 && (j & (C::DUP - 1)) != 0) {
+#pragma unroll
+            for (int f = 0; f < C::NFIN; ++f) l_f[f] = 0.f;  // a copy of another lane's sums
         }
-        const int lblk = blk0 + warp + k * kDecodeWarps;
-        const int n_valid = ((bad_mask >> s) & 1u) ? 0 : (lblk == nblk_seq - 1 ? last_valid : kBlockSize);
-        unsigned char *kb = ring + s * C::STAGE_BYTES;
-        unsigned char *vb = kb + kBlockSize * C::R;
-        if (n_valid < kBlockSize) {
-            if (n_valid == 0) {  // a table entry outside the pool: nothing of this block is used
-                __syncwarp();
-                if (issued < nb_w) issue(issued++);
-                continue;
-            }
-            // Rows past the context may hold anything (NaN included) and have
-            // probability 0: clear their V so that 0 * V adds nothing.
-            for (int i = n_valid * (C::R / 16) + lane; i < kBlockSize * (C::R / 16); i += 32)
-                reinterpret_cast<uint4 *>(vb)[i] = make_uint4(0u, 0u, 0u, 0u);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        float l_head[G], m_head[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float x = 0.f;
+#pragma unroll
+            for (int f = 0; f < C::NFIN; ++f) x += (g == hmask + f) ? l_f[f] : 0.f;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            l_head[g] = x;
+            m_head[g] = __shfl_sync(0xffffffffu, m_col, g);
         }
-
-        // ---- scores: q . k for the G heads, this lane's columns, steps in lane
-        // order. Step slots s and s + STEPS/2 meet at the first reduce step, so
-        // they are computed together and reduced at once (fewer live partials).
-        auto qk_step = [&](int st, float (&a)[G]) {
-            const int row = (st ^ smask) * C::RS + rg;
-            f32x2 s2[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) s2[g] = 0ull;
-#pragma unroll
-            for (int ch = 0; ch < C::CH; ++ch) {
-                f32x2 k2[VP];
-                load_chunk<Tc, C::CB>(kb + row * C::R + (ch * C::L + j) * C::CB, k2);
-#pragma unroll
-                for (int e = 0; e < VP; ++e)
-#pragma unroll
-                    for (int g = 0; g < G; ++g) fma2(s2[g], q2[g][ch * VP + e], k2[e]);
-            }
+        const long long u_lo = s_lo + cc.r - cc.blk, u_hi = u_lo + cc.nblk;  // the unit's positions
+        const bool whole = u_lo >= s_lo && u_hi <= s_hi;
+        const int u = cc.b * Hk + cc.hk;
+        const size_t slot = static_cast<size_t>(slice) + u;
+        if (rg == 0) {  // lanes of row group 0 hold the warp's O for their columns
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float a0, a1;
-                unpack2(s2[g], a0, a1);
-                a[g] = a0 + a1;
+                const int d0 = j * C::VE;
+                const float sc = whole ? (l_head[g] > 0.f ? prm.v_scale / l_head[g] : 0.f) : prm.v_scale;
+#pragma unroll
+                for (int e = 0; e < VP; e += 2) {
+                    float x0, x1, x2, x3;
+                    unpack2(acc2[g][e], x0, x1);
+                    unpack2(acc2[g][e + 1], x2, x3);
+                    const float4 o = make_float4(x0 * sc, x1 * sc, x2 * sc, x3 * sc);
+                    if (whole) {
+                        store_out4(static_cast<Tq *>(prm.out) +
+                                       (static_cast<size_t>(cc.b) * prm.num_heads + cc.hk * G + g) * D + d0 + 2 * e,
+                                   o);
+                    } else {
+                        *reinterpret_cast<float4 *>(prm.ws_o + (slot * G + g) * D + d0 + 2 * e) = o;
+                    }
+                }
             }
-        };
-        float part[C::NPART / 2];
-#pragma unroll
-        for (int st = 0; st < C::STEPS / 2; ++st) {
-            float lo[G], hi[G];
-            qk_step(st, lo);
-            qk_step(st + C::STEPS / 2, hi);
-#pragma unroll
-            for (int g = 0; g < G; ++g) part[st * G + g] = lo[g] + __shfl_xor_sync(0xffffffffu, hi[g], C::L / 2);
         }
-        TransposeReduce<C::NPART / 2, C::L / 4>::run(part);
-        float sc[C::NFIN];
+        if (!whole && lane < G) {
+            float m = m_head[0], l = l_head[0];
 #pragma unroll
-        for (int f = 0; f < C::NFIN; ++f) sc[f] = part[f];
-        if (n_valid < kBlockSize && t_own >= n_valid) {
-#pragma unroll
-            for (int f = 0; f < C::NFIN; ++f) sc[f] = -CUDART_INF_F;
+            for (int g = 1; g < G; ++g)
+                if (lane == g) {
+                    m = m_head[g];
+                    l = l_head[g];
+                }
+            prm.ws_m[slot * G + lane] = m;
+            prm.ws_l[slot * G + lane] = l;
         }
+        if (lane == 0 && u_lo >= s_lo) {  // the unit starts in this slice: where its partials are
+            int *rec = prm.ws_unit + 2 * static_cast<size_t>(u);
+            rec[0] = slice;
+            rec[1] = whole ? 1 : slice_of(u_hi - 1, N, WS) - slice + 1;
+        }
+    };
 
-        // ---- online softmax. The max of a head moves (and O, l are rescaled)
-        // only when one of its scores exceeds it by more than 8 (a factor 256
-        // in probability); otherwise the older max is kept and P stays below
-        // 2^8. The result is the same softmax, with fewer rescales.
-        bool grow = false;
-#pragma unroll
-        for (int f = 0; f < C::NFIN; ++f) grow |= sc[f] > thr_f[f];
-        if (__any_sync(0xffffffffu, grow)) {
-            // Block maxima through the buffer: scores in, one head per lane column.
-#pragma unroll
-            for (int f = 0; f < C::NFIN; ++f) pbuf[(t_own * G + hmask + f) * 2] = sc[f];
-            __syncwarp();
-            constexpr int ENT = (kBlockSize * G + 31) / 32;
-            float mx = -CUDART_INF_F;
-#pragma unroll
-            for (int e = 0; e < ENT; ++e) {
-                const int idx = lane + 32 * e;
-                if (idx < kBlockSize * G) mx = fmaxf(mx, pbuf[idx * 2]);
-            }
-#pragma unroll
-            for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float m_new = fmaxf(m_col, mx);
-            const float alpha = m_new == -CUDART_INF_F ? 1.f : exp2f(m_col - m_new);
-            m_col = m_new;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {  // lane g holds head g's values
-                const float a = __shfl_sync(0xffffffffu, alpha, g);
-                const f32x2 a2 = pack2(a, a);
-#pragma unroll
-                for (int e = 0; e < P2; ++e) mul2(acc2[g][e], a2);
-            }
-#pragma unroll
-            for (int f = 0; f < C::NFIN; ++f) {
-                const float mf = __shfl_sync(0xffffffffu, m_col, hmask + f);
-                l_f[f] *= __shfl_sync(0xffffffffu, alpha, hmask + f);
-                mu_f[f] = mf == -CUDART_INF_F ? 0.f : mf;
-                thr_f[f] = mf + 8.f;
-            }
-            __syncwarp();  // every lane has read the scores before they are overwritten
+    reset_state();
+    bool need_q = true;
+    int k = 0;
+    for (; k < nb_w; ++k) {
+        if (need_q) {
+            load_q(cc.b, cc.hk);
+            need_q = false;
         }
-        // probabilities, stored as (p, p) pairs for the packed P.V
-        if constexpr (C::NFIN == 1) {
-            const float p0 = ex2_approx(sc[0] - mu_f[0]);
-            l_f[0] += p0;
-            asm volatile("st.shared.v2.f32 [%0], {%1, %1};" ::"r"(p_own), "f"(p0) : "memory");
-        } else {
-#pragma unroll
-            for (int f = 0; f < C::NFIN; f += 2) {
-                const float p0 = ex2_approx(sc[f] - mu_f[f]);
-                const float p1 = ex2_approx(sc[f + 1] - mu_f[f + 1]);
-                l_f[f] += p0;
-                l_f[f + 1] += p1;
-                asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(p_own + f * 8), "f"(p0), "f"(p1)
-                             : "memory");
+        const int s = k % C::NSTAGE;
+        const bool landed = mbar_wait(bars + 8 * s, (k / C::NSTAGE) & 1);
+        if (!__all_sync(0xffffffffu, landed)) break;
+        const int last_valid = cc.c - (cc.nblk - 1) * kBlockSize;
+        const int n_valid = ((bad_mask >> s) & 1u) ? 0 : (cc.blk == cc.nblk - 1 ? last_valid : kBlockSize);
+        unsigned char *kb = ring + s * C::STAGE_BYTES;
+        unsigned char *vb = kb + kBlockSize * C::R;
+        if (n_valid > 0) {
+            if (n_valid < kBlockSize) {
+                // Rows past the context may hold anything (NaN included) and have
+                // probability 0: clear their V so that 0 * V adds nothing.
+                for (int i = n_valid * (C::R / 16) + lane; i < kBlockSize * (C::R / 16); i += 32)
+                    reinterpret_cast<uint4 *>(vb)[i] = make_uint4(0u, 0u, 0u, 0u);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-        }
-        __syncwarp();
 
-        // ---- O += P . V
+            // ---- scores: q . k for the G heads, this lane's columns, steps in lane
+            // order. Step slots s and s + STEPS/2 meet at the first reduce step, so
+            // they are computed together and reduced at once (fewer live partials).
+            auto qk_step = [&](int st, float(&a)[G]) {
+                const int row = (st ^ smask) * C::RS + rg;
+                f32x2 s2[G];
 #pragma unroll
-        for (int st = 0; st < C::STEPS; ++st) {
-            const int t = st * C::RS + rg;
-            f32x2 pr[G];
-            if constexpr (G == 1) {
-                pr[0] = lds_pair(pbuf_s + t * 8);
+                for (int g = 0; g < G; ++g) s2[g] = 0ull;
+#pragma unroll
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    f32x2 k2[VP];
+                    load_chunk<Tc, C::CB>(kb + row * C::R + (ch * C::L + j) * C::CB, k2);
+#pragma unroll
+                    for (int e = 0; e < VP; ++e)
+#pragma unroll
+                        for (int g = 0; g < G; ++g) fma2(s2[g], q2[g][ch * VP + e], k2[e]);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float a0, a1;
+                    unpack2(s2[g], a0, a1);
+                    a[g] = a0 + a1;
+                }
+            };
+            float part[C::NPART / 2];
+#pragma unroll
+            for (int st = 0; st < C::STEPS / 2; ++st) {
+                float lo[G], hi[G];
+                qk_step(st, lo);
+                qk_step(st + C::STEPS / 2, hi);
+#pragma unroll
+                for (int g = 0; g < G; ++g) part[st * G + g] = lo[g] + __shfl_xor_sync(0xffffffffu, hi[g], C::L / 2);
+            }
+            TransposeReduce<C::NPART / 2, C::L / 4>::run(part);
+            float sc[C::NFIN];
+#pragma unroll
+            for (int f = 0; f < C::NFIN; ++f) sc[f] = part[f];
+            if (n_valid < kBlockSize && t_own >= n_valid) {
+#pragma unroll
+                for (int f = 0; f < C::NFIN; ++f) sc[f] = -CUDART_INF_F;
+            }
+
+            // ---- online softmax. The max of a head moves (and O, l are rescaled)
+            // only when one of its scores exceeds it by more than 8 (a factor 256
+            // in probability); otherwise the older max is kept and P stays below
+            // 2^8. The result is the same softmax, with fewer rescales.
+            bool grow = false;
+#pragma unroll
+            for (int f = 0; f < C::NFIN; ++f) grow |= sc[f] > thr_f[f];
+            if (__any_sync(0xffffffffu, grow)) {
+                // Block maxima through the buffer: scores in, one head per lane column.
+#pragma unroll
+                for (int f = 0; f < C::NFIN; ++f) pbuf[(t_own * G + hmask + f) * 2] = sc[f];
+                __syncwarp();
+                constexpr int ENT = (kBlockSize * G + 31) / 32;
+                float mx = -CUDART_INF_F;
+#pragma unroll
+                for (int e = 0; e < ENT; ++e) {
+                    const int idx = lane + 32 * e;
+                    if (idx < kBlockSize * G) mx = fmaxf(mx, pbuf[idx * 2]);
+                }
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float m_new = fmaxf(m_col, mx);
+                const float alpha = m_new == -CUDART_INF_F ? 1.f : exp2f(m_col - m_new);
+                m_col = m_new;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {  // lane g holds head g's values
+                    const float a = __shfl_sync(0xffffffffu, alpha, g);
+                    const f32x2 a2 = pack2(a, a);
+#pragma unroll
+                    for (int e = 0; e < P2; ++e) mul2(acc2[g][e], a2);
+                }
+#pragma unroll
+                for (int f = 0; f < C::NFIN; ++f) {
+                    const float mf = __shfl_sync(0xffffffffu, m_col, hmask + f);
+                    l_f[f] *= __shfl_sync(0xffffffffu, alpha, hmask + f);
+                    mu_f[f] = mf == -CUDART_INF_F ? 0.f : mf;
+                    thr_f[f] = mf + 8.f;
+                }
+                __syncwarp();  // every lane has read the scores before they are overwritten
+            }
+            // probabilities, stored as (p, p) pairs for the packed P.V
+            if constexpr (C::NFIN == 1) {
+                const float p0 = ex2_approx(sc[0] - mu_f[0]);
+                l_f[0] += p0;
+                asm volatile("st.shared.v2.f32 [%0], {%1, %1};" ::"r"(p_own), "f"(p0) : "memory");
             } else {
 #pragma unroll
-                for (int g = 0; g < G; g += 2) lds_pair2(pbuf_s + (t * G + g) * 8, pr[g], pr[g + 1]);
+                for (int f = 0; f < C::NFIN; f += 2) {
+                    const float p0 = ex2_approx(sc[f] - mu_f[f]);
+                    const float p1 = ex2_approx(sc[f + 1] - mu_f[f + 1]);
+                    l_f[f] += p0;
+                    l_f[f + 1] += p1;
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %1, %2, %2};" ::"r"(p_own + f * 8), "f"(p0),
+                                 "f"(p1)
+                                 : "memory");
+                }
             }
+            __syncwarp();
+
+            // ---- O += P . V
 #pragma unroll
-            for (int ch = 0; ch < C::CH; ++ch) {
-                f32x2 v2[VP];
-                load_chunk<Tc, C::CB>(vb + t * C::R + (ch * C::L + j) * C::CB, v2);
+            for (int st = 0; st < C::STEPS; ++st) {
+                const int t = st * C::RS + rg;
+                f32x2 pr[G];
+                if constexpr (G == 1) {
+                    pr[0] = lds_pair(pbuf_s + t * 8);
+                } else {
 #pragma unroll
-                for (int e = 0; e < VP; ++e)
+                    for (int g = 0; g < G; g += 2) lds_pair2(pbuf_s + (t * G + g) * 8, pr[g], pr[g + 1]);
+                }
 #pragma unroll
-                    for (int g = 0; g < G; ++g) fma2(acc2[g][ch * VP + e], pr[g], v2[e]);
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    f32x2 v2[VP];
+                    load_chunk<Tc, C::CB>(vb + t * C::R + (ch * C::L + j) * C::CB, v2);
+#pragma unroll
+                    for (int e = 0; e < VP; ++e)
+#pragma unroll
+                        for (int g = 0; g < G; ++g) fma2(acc2[g][ch * VP + e], pr[g], v2[e]);
+                }
             }
         }
         __syncwarp();
-        if (issued < nb_w) {
-            issue(issued);
-            if (C::PF > 0) prefetch(issued + C::PF, issued);
-            ++issued;
+        Cursor nx = cc;  // this warp's next block
+        const int passed = k + 1 < nb_w ? cursor_advance(nx, 1, prm) : 0;
+        if (k + C::NSTAGE < nb_w) {
+            Cursor ic = nx;
+            cursor_advance(ic, C::NSTAGE - 1, prm);
+            issue(k + C::NSTAGE, ic);
         }
-    }
-    if (failed) {
-        // Let copies still in flight land before the ring is reused.
-        for (int kk = k; kk < issued; ++kk) mbar_wait(bars + 8 * (kk % C::NSTAGE), (kk / C::NSTAGE) & 1);
-    }
-
-    // ---- merge the warps (and each warp's row groups) of this CTA
-    if (C::DUP > 1 && (j & (C::DUP - 1)) != 0) {
-#pragma unroll
-        for (int f = 0; f < C::NFIN; ++f) l_f[f] = 0.f;  // a copy of another lane's sums
-    }
-    float l_head[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float x = 0.f;
-#pragma unroll
-        for (int f = 0; f < C::NFIN; ++f) x += (g == hmask + f) ? l_f[f] : 0.f;
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        l_head[g] = x;
-    }
-    __syncthreads();
-    float *red_acc = reinterpret_cast<float *>(smem);  // [warp][rg][g][D]
-    float *red_m = reinterpret_cast<float *>(smem + C::OFF_ML);
-    float *red_l = red_m + kDecodeWarps * G;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float mg = __shfl_sync(0xffffffffu, m_col, g);
-        if (lane == 0) {
-            red_m[warp * G + g] = mg;
-            red_l[warp * G + g] = l_head[g];
+        // ---- the last block, or the next one in another unit: the segment closes
+        if (passed > 0 || k + 1 == nb_w) {
+            close_segment();
+            reset_state();
+            need_q = true;
         }
+        cc = nx;
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int ch = 0; ch < C::CH; ++ch) {
-            float *dst = red_acc + ((warp * C::RS + rg) * G + g) * D + (ch * C::L + j) * C::VE;
-#pragma unroll
-            for (int e = 0; e < VP; e += 2) {
-                float x0, x1, x2, x3;
-                unpack2(acc2[g][ch * VP + e], x0, x1);
-                unpack2(acc2[g][ch * VP + e + 1], x2, x3);
-                *reinterpret_cast<float4 *>(dst + 2 * e) = make_float4(x0, x1, x2, x3);
-            }
-        }
-    __syncthreads();
-
-    for (int idx = threadIdx.x; idx < G * D; idx += kDecodeThreads) {
-        const int g = idx / D, d = idx % D;
-        float M = -CUDART_INF_F;
-#pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, red_m[w * G + g]);
-        float O = 0.f, Lsum = 0.f;
-        if (M != -CUDART_INF_F) {
-#pragma unroll
-            for (int w = 0; w < kDecodeWarps; ++w) {
-                const float mw = red_m[w * G + g];
-                if (mw == -CUDART_INF_F) continue;
-                const float wt = exp2f(mw - M);
-                float o = 0.f;
-#pragma unroll
-                for (int r = 0; r < C::RS; ++r) o += red_acc[((w * C::RS + r) * G + g) * D + d];
-                O += wt * o;
-                Lsum += wt * red_l[w * G + g];
-            }
-        }
-        O *= prm.v_scale;
-        const int h = hk * G + g;
-        if (parts == 1) {
-            Tq *out = static_cast<Tq *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + h) * D + d;
-            store_out(out, Lsum > 0.f ? O / Lsum : 0.f);
-        } else {
-            const size_t pi = (static_cast<size_t>(b) * prm.num_heads + h) * prm.max_parts + p;
-            prm.ws_o[pi * D + d] = O;
-            if (d == 0) {
-                prm.ws_m[pi] = M;
-                prm.ws_l[pi] = Lsum;
-            }
-        }
+    if (k < nb_w) {
+        // A bounded wait gave up (the status word says why): let copies still in
+        // flight land before the CTA ends.
+        for (int kk = k; kk < min(k + C::NSTAGE, nb_w); ++kk)
+            mbar_wait(bars + 8 * (kk % C::NSTAGE), (kk / C::NSTAGE) & 1);
     }
-    if (parts == 1 || !prm.fuse_merge) return;
-
-    // ---- fused merge: the last CTA of this (sequence, KV head) to finish merges
-    // every partition's partials. Partials are published (fence) before the
-    // ticket is taken, and read from L2 after it. A ticket is the call's stamp
-    // and the arrivals so far; one with another stamp (an earlier call, or
-    // memory never used as a ticket) counts as no arrivals, so the workspace
-    // needs no initialisation.
-    int *flag = reinterpret_cast<int *>(smem + C::OFF_FLAG);
-    unsigned long long *ticket = prm.ws_ticket + static_cast<size_t>(b) * prm.num_kv_heads + hk;
-    const unsigned long long stamp = static_cast<unsigned long long>(prm.stamp) << 32;
-    __syncthreads();  // the CTA's partial writes happen before thread 0's fence (cumulativity)
-    if (threadIdx.x == 0) {
-        __threadfence();
-        unsigned long long cur = __ldcg(ticket), seen;
-        unsigned int n;
-        do {
-            seen = cur;
-            n = (seen & 0xffffffff00000000ull) == stamp ? static_cast<unsigned int>(seen) : 0u;
-            cur = atomicCAS(ticket, seen, stamp | (n + 1u));
-        } while (cur != seen);
-        if (n >= static_cast<unsigned int>(parts)) flag_status(PA_STATUS_BAD_WORKSPACE);
-        *flag = n + 1u == static_cast<unsigned int>(parts);
-    }
-    __syncthreads();
-    if (!*flag) return;
-    __threadfence();
-    merge_partitions_n<Tq, (G * D + kDecodeThreads - 1) / kDecodeThreads>(prm, b, hk * G, threadIdx.x,
-                                                                          kDecodeThreads, G * D, parts, D);
-    if (threadIdx.x == 0) atomicExch(ticket, stamp);  // no arrivals: a replay of this call starts afresh
 }
 
-// Merge the partitions of every sequence that has more than one (the merge of
-// pa_decode_merge, a kernel of its own). Grid (KV head, sequence), G * D
-// threads: one per output element of the group. It is launched as a
-// programmatic dependent of decode_kernel and waits for it
-// (griddepcontrol.wait) before reading the partials.
-template <typename T>
-__global__ void decode_reduce_kernel(const DecodeParams prm, int D) {
-    // context_lens was written before decode_kernel ran (decode_kernel waited for
-    // it), so it may be read before waiting for decode_kernel's partials.
-    const int hk = blockIdx.x, b = blockIdx.y;
-    const int G = prm.num_heads / prm.num_kv_heads;
-    const int g = threadIdx.x / D, d = threadIdx.x % D;
-    const int cap = min(prm.max_blocks_per_seq * kBlockSize, prm.max_context_len);
-    const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
-    const int parts = max(1, (c + prm.part_tokens - 1) / prm.part_tokens);
-    if (parts == 1 || g >= G) return;
+// Merge the partials of every unit cut by slice boundaries:
+//   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L
+// over the unit's slices s (slots first + u .. first + slices - 1 + u). Grid
+// (units, G*D/128 column groups); a thread takes four consecutive columns of one
+// head, with every slot's loads of a round in flight together (up to 8 slots a
+// round). A programmatic dependent of decode_kernel: it waits for it before
+// reading the workspace.
+template <typename T, int G, int D>
+__global__ void __launch_bounds__(32) decode_merge_kernel(const DecodeParams prm) {
+    const int u = blockIdx.x;
+    const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
+    const int idx = 4 * (blockIdx.y * 32 + threadIdx.x);
+    if (idx >= G * D) return;
+    if (clamp_context(__ldg(prm.context_lens + b), decode_cap(prm), false) == 0) return;  // zero rows, written
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    merge_partitions<T>(prm, b, hk * G + g, parts, d, D);
+    const int first = __ldcg(prm.ws_unit + 2 * u), nseg = __ldcg(prm.ws_unit + 2 * u + 1);
+    if (nseg <= 1) return;  // a whole unit: written by the decode kernel
+    const int g = idx / D, d = idx % D;
+    const int s0 = first + u;
+    float M = -CUDART_INF_F, Lsum = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < nseg; p0 += 8) {
+        float mp[8], lp[8];
+        float4 op[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool in = p0 + i < nseg;
+            const size_t s = static_cast<size_t>(s0 + p0 + i);
+            mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
+            lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
+            op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mc = M;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
+        if (mc == -CUDART_INF_F) continue;
+        const float a = exp2f(M - mc);  // 0 while M is still -inf
+        O.x *= a;
+        O.y *= a;
+        O.z *= a;
+        O.w *= a;
+        Lsum *= a;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (mp[i] == -CUDART_INF_F) continue;  // a slice whose blocks were all skipped
+            const float wt = exp2f(mp[i] - mc);
+            O.x += wt * op[i].x;
+            O.y += wt * op[i].y;
+            O.z += wt * op[i].z;
+            O.w += wt * op[i].w;
+            Lsum += wt * lp[i];
+        }
+        M = mc;
+    }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    O.x *= inv;
+    O.y *= inv;
+    O.z *= inv;
+    O.w *= inv;
+    store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
 }
 
 }  // namespace pa

@@ -66,113 +66,103 @@ int check_shape(const pa_shape *s) {
 int elem_bytes(const pa_shape *s) { return s->dtype == PA_DTYPE_BF16 ? 2 : 4; }
 int cache_elem_bytes(const pa_shape *s) { return s->kv_fp8 ? 1 : elem_bytes(s); }
 
-// Tokens per split-context partition. A context of at most one partition is
-// handled by the single pass alone (no workspace, no reduce kernel).
-// Automatic split-context partition length. A (sequence, KV head) unit is one
-// CTA per partition, and `slots` decode CTAs are resident at once. Splitting
-// balances the tail of unequal lengths but costs partial writes and the merge,
-// so: no split when the units alone fill the GPU four times over; otherwise the
-// longest power of two from 512 to 4096 tokens that still gives about four
-// waves; and for small batches shorter partitions (down to 128) so the grid
-// still covers the GPU. Measured on B200: 256 sequences of 1.5-2 K tokens run
-// 17 % faster unsplit than at 512; 8 x 32 K tokens 3 % faster at 1024.
-int partition_tokens(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s) {
-    if (requested > 0) return requested;
-    const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
-    const int64_t sms = sm_count() > 0 ? sm_count() : 148;
-    const int64_t slots = sms * (s->num_heads / s->num_kv_heads <= 4 ? 3 : 2);  // resident decode CTAs
-    const int whole = max(64, ((max_context_len + 63) / 64) * 64);
-    if (units >= 4 * slots) return whole;
-    auto parts = [&](int tp) -> int64_t { return (max_context_len + tp - 1) / tp; };
-    int tp = 512;
-    while (tp < 4096 && units * parts(2 * tp) >= 4 * slots) tp *= 2;
-    while (tp > 128 && units * parts(tp) < 2 * sms) tp /= 2;
-    return max_context_len <= tp ? whole : tp;
+// CTAs of the decode kernel one SM holds, for this shape: the occupancy the
+// runtime reports on the current device (with the kernel's shared memory and
+// the largest shared-memory carveout, set here once per device), or, without
+// a device, the compile-time estimate. The grid is sized from it, so every
+// slice's CTA is resident from the start.
+template <typename Tq, typename Tc, int D, int G>
+int resident_of() {
+    using C = pa::DecodeCfg<Tc, D, G>;
+    static std::atomic<int> cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return C::RESIDENT;
+    }
+    int n = cached[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
+    auto kernel = pa::decode_kernel<Tq, Tc, D, G>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, pa::kDecodeThreads, C::SMEM) != cudaSuccess ||
+        n < 1) {
+        cudaGetLastError();
+        return C::RESIDENT;
+    }
+    cached[dev].store(n, std::memory_order_release);
+    return n;
+}
+
+template <typename Tq, typename Tc, int D>
+int resident_g(int g) {
+    switch (g) {
+        case 1: return resident_of<Tq, Tc, D, 1>();
+        case 2: return resident_of<Tq, Tc, D, 2>();
+        case 4: return resident_of<Tq, Tc, D, 4>();
+        default: return resident_of<Tq, Tc, D, 8>();
+    }
+}
+
+int decode_resident(const pa_shape *s) {
+    const int g = s->num_heads / s->num_kv_heads;
+    if (s->kv_fp8)
+        return s->head_dim == 128 ? resident_g<__nv_bfloat16, pa::fp8e4m3, 128>(g)
+                                  : resident_g<__nv_bfloat16, pa::fp8e4m3, 64>(g);
+    if (s->dtype == PA_DTYPE_BF16)
+        return s->head_dim == 128 ? resident_g<__nv_bfloat16, __nv_bfloat16, 128>(g)
+                                  : resident_g<__nv_bfloat16, __nv_bfloat16, 64>(g);
+    return s->head_dim == 128 ? resident_g<float, float, 128>(g) : resident_g<float, float, 64>(g);
 }
 
 struct DecodeGeometry {
-    int part_tokens;
-    int max_parts;
-    int64_t ws_bytes;
+    int ctas;          // grid of the persistent decode kernel (kDecodeWarps slices each)
+    int64_t slots;     // partial (m, l, O) slots: slice index + unit index
+    int64_t ws_bytes;  // workspace bytes
 };
 
 int64_t round16(int64_t n) { return (n + 15) / 16 * 16; }
 
-// Workspace layout (split contexts only): fp32 O [B][H][P][D], then m and l
-// [B][H][P], then the fused merge's 64-bit tickets [B][Hk]; each 16-byte aligned.
+// The decode kernel cuts the flat (sequence, KV head, block) list into
+// 4 * ctas equal slices, one per warp. Automatic: the CTAs all SMs hold at once
+// (each warp streams one slice; balance comes from equal slices, not from many
+// waves), but no more than one warp per 4 blocks of the largest possible list.
+// With partition_tokens given: slices of about that many tokens of a context
+// of max_context_len. Workspace: fp32 partial outputs [slots][G][D], partial
+// maxima and sums [slots][G] each, then int32 (first slice, slices) records
+// [B][Hk]; each part 16-byte aligned.
 int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s,
                     DecodeGeometry *g) {
     if (num_seqs < 0 || max_context_len < 0) return PA_ERR_INVALID_ARGUMENT;
     if (requested < 0 || (requested > 0 && (requested % 64 != 0))) return PA_ERR_INVALID_ARGUMENT;
-    g->part_tokens = partition_tokens(num_seqs, max_context_len, requested, s);
-    g->max_parts = max_context_len > 0 ? (max_context_len + g->part_tokens - 1) / g->part_tokens : 1;
-    if (g->max_parts < 1) g->max_parts = 1;
-    if (g->max_parts == 1) {
+    const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
+    const int64_t n_max = units * ((max_context_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+    int64_t slices;
+    if (requested > 0) {
+        slices = (n_max * PA_BLOCK_SIZE + requested - 1) / requested;
+    } else {
+        const int64_t sms = sm_count() > 0 ? sm_count() : 148;
+        slices = std::min<int64_t>(sms * decode_resident(s) * pa::kDecodeWarps, (n_max + 3) / 4);
+    }
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>((slices + pa::kDecodeWarps - 1) / pa::kDecodeWarps,
+                                                                  65535));
+    g->ctas = static_cast<int>(ctas);
+    if (units == 0) {
+        g->slots = 0;
         g->ws_bytes = 0;
     } else {
-        const int64_t n = static_cast<int64_t>(num_seqs) * s->num_heads * g->max_parts;
-        const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
-        g->ws_bytes = n * s->head_dim * 4 + round16(n * 4) * 2 + round16(units * 8);
+        const int gq = s->num_heads / s->num_kv_heads;
+        g->slots = ctas * pa::kDecodeWarps + units - 1;
+        g->ws_bytes = g->slots * gq * s->head_dim * 4 + round16(g->slots * gq * 4) * 2 + round16(units * 8);
     }
     return PA_OK;
 }
-
-// Opt a kernel into `bytes` of dynamic shared memory, once per device.
-template <typename K>
-int allow_smem(K kernel, int bytes, std::atomic<uint64_t> &done) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e);
-    const uint64_t bit = uint64_t{1} << (dev & 63);
-    if (done.load(std::memory_order_acquire) & bit) return PA_OK;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return cuda_fail(e);
-    done.fetch_or(bit, std::memory_order_acq_rel);
-    return PA_OK;
-}
-
-// A stamp per launch for the fused merge's tickets: nonzero (a zeroed
-// workspace holds stamp 0) and different from the stamps of recent launches.
-// A launch captured in a CUDA graph keeps its stamp on every replay; its last
-// CTAs put the tickets back to (stamp, 0), so replays start afresh too.
-uint32_t next_stamp() {
-    static std::atomic<uint32_t> counter{0};
-    uint32_t s;
-    do {
-        s = counter.fetch_add(1, std::memory_order_relaxed) + 1;
-    } while (s == 0);
-    return s;
-}
-
-// pa_decode: the split-context kernel with the merge fused into it.
-// pa_decode_partitions / pa_decode_merge: the split-context kernel without the
-// fused merge, and the merge as a kernel of its own.
-enum DecodeMode { kDecodeFused, kDecodePartitions, kDecodeMerge };
 
 template <typename Tq, typename Tc, int D, int G>
-int launch_decode(pa::DecodeParams prm, int num_seqs, cudaStream_t st, DecodeMode mode) {
+int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaStream_t st) {
     using C = pa::DecodeCfg<Tc, D, G>;
-    // Both kernels are programmatic dependent launches: each starts launching
-    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
-    // before reading anything.
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (mode == kDecodeMerge) {
-        if (prm.max_parts == 1) return PA_OK;  // no context is split
-        cfg.gridDim = dim3(prm.num_kv_heads, num_seqs);
-        cfg.blockDim = dim3(G * D);
-        cfg.dynamicSmemBytes = 0;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_reduce_kernel<Tq>, prm, D);
-        return e == cudaSuccess ? PA_OK : cuda_fail(e);
-    }
-    static std::atomic<uint64_t> smem_done{0};
-    int arc = allow_smem(pa::decode_kernel<Tq, Tc, D, G>, C::SMEM, smem_done);
-    if (arc != PA_OK) return arc;
+    resident_of<Tq, Tc, D, G>();  // sets the kernel's shared-memory attributes on this device
     CUtensorMap tm_k{}, tm_v{};
     const uint64_t rows = static_cast<uint64_t>(prm.num_blocks) * pa::kBlockSize;
     if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
@@ -180,22 +170,35 @@ int launch_decode(pa::DecodeParams prm, int num_seqs, cudaStream_t st, DecodeMod
         !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
         return PA_ERR_UNSUPPORTED;
-    prm.fuse_merge = mode == kDecodeFused ? 1 : 0;
-    prm.stamp = next_stamp();
-    cfg.gridDim = dim3(prm.num_kv_heads, num_seqs, prm.max_parts);
+    // Both kernels are programmatic dependent launches: each starts launching
+    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
+    // before reading what it wrote.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(geo.ctas);
     cfg.blockDim = dim3(pa::kDecodeThreads);
     cfg.dynamicSmemBytes = C::SMEM;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cfg.gridDim = dim3(static_cast<unsigned>(prm.num_seqs) * prm.num_kv_heads, (G * D + 127) / 128);
+    cfg.blockDim = dim3(32);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D>, prm);
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
 template <typename Tq, typename Tc, int D>
-int dispatch_g(int g, const pa::DecodeParams &prm, int num_seqs, cudaStream_t st, DecodeMode mode) {
+int dispatch_g(int g, const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaStream_t st) {
     switch (g) {
-        case 1: return launch_decode<Tq, Tc, D, 1>(prm, num_seqs, st, mode);
-        case 2: return launch_decode<Tq, Tc, D, 2>(prm, num_seqs, st, mode);
-        case 4: return launch_decode<Tq, Tc, D, 4>(prm, num_seqs, st, mode);
-        case 8: return launch_decode<Tq, Tc, D, 8>(prm, num_seqs, st, mode);
+        case 1: return launch_decode<Tq, Tc, D, 1>(prm, geo, st);
+        case 2: return launch_decode<Tq, Tc, D, 2>(prm, geo, st);
+        case 4: return launch_decode<Tq, Tc, D, 4>(prm, geo, st);
+        case 8: return launch_decode<Tq, Tc, D, 8>(prm, geo, st);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -267,10 +270,11 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
 
 namespace {
 
-int decode_stages(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-                  int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
-                  float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
-                  const pa_shape *shape, void *stream, DecodeMode mode) {
+// pa_decode after its argument checks.
+int decode_call(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
+                float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
+                const pa_shape *shape, void *stream) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -280,20 +284,22 @@ int decode_stages(void *out, const void *q, const void *k_cache, const void *v_c
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned(block_tables, 4) ||
         !aligned(context_lens, 4))
         return PA_ERR_ALIGNMENT;
+    if (static_cast<int64_t>(num_seqs) * shape->num_kv_heads > 0x7fffffff) return PA_ERR_UNSUPPORTED;
     DecodeGeometry g;
     rc = decode_geometry(num_seqs, max_context_len, partition_tokens, shape, &g);
     if (rc != PA_OK) return rc;
-    if (num_seqs > 65535 || g.max_parts > 65535) return PA_ERR_UNSUPPORTED;  // grid y / z limits
     pa::DecodeParams prm{};
-    if (g.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < g.ws_bytes) return PA_ERR_WORKSPACE;
-        if (!aligned16(workspace)) return PA_ERR_ALIGNMENT;
-        const int64_t n = static_cast<int64_t>(num_seqs) * shape->num_heads * g.max_parts;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!workspace || workspace_bytes < g.ws_bytes) return PA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return PA_ERR_ALIGNMENT;
+    {
+        const int gq = shape->num_heads / shape->num_kv_heads;
         char *w = static_cast<char *>(workspace);
+        const int64_t o_bytes = g.slots * gq * shape->head_dim * 4, ml_bytes = round16(g.slots * gq * 4);
         prm.ws_o = reinterpret_cast<float *>(w);
-        prm.ws_m = reinterpret_cast<float *>(w + n * shape->head_dim * 4);
-        prm.ws_l = reinterpret_cast<float *>(w + n * shape->head_dim * 4 + round16(n * 4));
-        prm.ws_ticket = reinterpret_cast<unsigned long long *>(w + n * shape->head_dim * 4 + round16(n * 4) * 2);
+        prm.ws_m = reinterpret_cast<float *>(w + o_bytes);
+        prm.ws_l = reinterpret_cast<float *>(w + o_bytes + ml_bytes);
+        prm.ws_unit = reinterpret_cast<int *>(w + o_bytes + 2 * ml_bytes);
     }
     prm.out = out;
     prm.q = q;
@@ -302,12 +308,11 @@ int decode_stages(void *out, const void *q, const void *k_cache, const void *v_c
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
     prm.num_blocks = shape->num_blocks;
+    prm.num_seqs = num_seqs;
     prm.max_blocks_per_seq = max_blocks_per_seq;
     prm.num_heads = shape->num_heads;
     prm.num_kv_heads = shape->num_kv_heads;
     prm.max_context_len = max_context_len;
-    prm.part_tokens = g.part_tokens;
-    prm.max_parts = g.max_parts;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.v_scale = 1.f;
     if (shape->kv_fp8) {
@@ -315,18 +320,16 @@ int decode_stages(void *out, const void *q, const void *k_cache, const void *v_c
         prm.v_scale = shape->v_scale;
     }
     const int G = shape->num_heads / shape->num_kv_heads;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (shape->kv_fp8) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, num_seqs, st, mode)
-                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, num_seqs, st, mode);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, g, st)
+                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, g, st);
     }
     if (shape->dtype == PA_DTYPE_BF16) {
-        return shape->head_dim == 128
-                   ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, num_seqs, st, mode)
-                   : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, num_seqs, st, mode);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, g, st)
+                                      : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, g, st);
     }
-    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, num_seqs, st, mode)
-                                  : dispatch_g<float, float, 64>(G, prm, num_seqs, st, mode);
+    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, g, st)
+                                  : dispatch_g<float, float, 64>(G, prm, g, st);
 }
 
 }  // namespace
@@ -337,27 +340,8 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
               float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes, const pa_shape *shape,
               void *stream) {
-    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kDecodeFused);
-}
-
-int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
-                         const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
-                         int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
-                         void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream) {
-    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kDecodePartitions);
-}
-
-int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
-                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
-                    int64_t workspace_bytes, const pa_shape *shape, void *stream) {
-    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                         max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream,
-                         kDecodeMerge);
+    return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -455,13 +439,12 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
         const int rc = noalloc_scratch(&scratch);
         if (rc != PA_OK) return rc;
     }
-    // The two-kernel form (split-context pass, then the merge kernel) keeps no
-    // state between calls in the scratch: nothing in it has to start at zero.
-    int rc = decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                           max_context_len, scale, partition_tokens, scratch, need, shape, stream, kDecodePartitions);
-    if (rc != PA_OK) return rc;
-    return decode_stages(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                         max_context_len, scale, partition_tokens, scratch, need, shape, stream, kDecodeMerge);
+    if (need == 0) return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                    num_seqs, max_context_len, scale, partition_tokens, nullptr, 0, shape, stream);
+    // Every partial and record a call reads, it has written first: no earlier
+    // call's contents matter.
+    return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       max_context_len, scale, partition_tokens, scratch, need, shape, stream);
 }
 
 static int launch_copy(void *dst, const void *src, const int64_t *pairs, int64_t num_pairs, int64_t src_blocks,

@@ -230,6 +230,16 @@ struct Widen<float> {
 __device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
 __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
 
+// Four consecutive outputs (p 16-byte aligned for fp32, 8-byte for bf16).
+__device__ __forceinline__ void store_out4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store_out4(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 r;
+    r.x = *reinterpret_cast<const uint32_t *>(&a);
+    r.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = r;
+}
+
 __device__ __forceinline__ float load_in(const float *p) { return *p; }
 __device__ __forceinline__ float load_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 

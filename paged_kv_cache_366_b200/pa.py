@@ -25,7 +25,6 @@ PA_STATUS_BAD_SLOT = 0x2
 PA_STATUS_BAD_CONTEXT = 0x4
 PA_STATUS_WAIT_TIMEOUT = 0x8
 PA_STATUS_BAD_QUERY = 0x10
-PA_STATUS_BAD_WORKSPACE = 0x20
 PA_ABI_VERSION = 4
 
 
@@ -46,7 +45,7 @@ class PaShape(ctypes.Structure):
 EXPORTED = [
     "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
     "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version", "pa_decode_noalloc",
-    "pa_copy_blocks", "pa_swap_blocks", "pa_decode_partitions", "pa_decode_merge",
+    "pa_copy_blocks", "pa_swap_blocks",
 ]
 
 PA_ERR_SCRATCH_LIMIT = -7
@@ -63,9 +62,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_decode_workspace_bytes.argtypes = [I32, I32, I32, SP]
     lib.pa_decode_workspace_bytes.restype = I64
-    for fn in (lib.pa_decode, lib.pa_decode_partitions, lib.pa_decode_merge):
-        fn.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
-        fn.restype = ctypes.c_int
+    lib.pa_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
+    lib.pa_decode.restype = ctypes.c_int
     lib.pa_prefill_chunk.argtypes = [P, P, P, P, P, I32, P, P, I32, I32, I32, F, SP, P]
     lib.pa_prefill_chunk.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, SP, P]
@@ -209,22 +207,6 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
               k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """Decode attention of one query token per sequence over its paged context."""
     _decode("pa_decode", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale)
-
-
-def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
-                         scale: float, partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None,
-                         stream=None, k_scale: float = 0.0, v_scale: float = 0.0) -> None:
-    """pa_decode's split-context pass alone (same arguments); pa_decode_merge completes it."""
-    _decode("pa_decode_partitions", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale)
-
-
-def pa_decode_merge(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
-                    partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-                    k_scale: float = 0.0, v_scale: float = 0.0) -> None:
-    """pa_decode's merge of the split-context partials (same arguments as pa_decode)."""
-    _decode("pa_decode_merge", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
             partition_tokens, workspace, stream, k_scale, v_scale)
 
 

@@ -72,3 +72,11 @@ def mixed_step_reference():
     kc, vc = oracle_written(case)
     ref = oracle.prefill(case.q, kc, vc, case.block_tables, case.cu_q_lens, case.context_lens, case.scale)
     return case, ref
+
+
+def decode_workspace(pa, num_seqs, max_context_len, k_cache, num_heads, partition_tokens=0, k_scale=0.0,
+                     v_scale=0.0):
+    """A workspace of the size pa_decode asks for (uninitialised: pa_decode needs none)."""
+    n = pa.pa_decode_workspace_bytes(num_seqs, max_context_len, partition_tokens,
+                                     pa.shape_of(k_cache, num_heads, k_scale, v_scale))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=k_cache.device)

@@ -47,37 +47,40 @@ def shape(**kw):
     return pa.PaShape(**d)
 
 
+def r16(n):
+    return (n + 15) // 16 * 16
+
+
+def ws_bytes(B, ctas, H=32, Hk=8, D=128):
+    """Workspace of a decode over `ctas` CTAs (4 slices each): partial O, m and l per slot (slice + unit),
+    then an int32 (first slice, slices) record per unit."""
+    units = B * Hk
+    slots = 4 * ctas + units - 1
+    g = H // Hk
+    return slots * g * D * 4 + 2 * r16(slots * g * 4) + r16(units * 8)
+
+
 def test_workspace_sizes():
     from paged_kv_cache_366_b200 import pa
     s = shape()
-    # single pass for short contexts: no workspace
-    assert pa.pa_decode_workspace_bytes(64, 300, 0, s) == 0
-    # split contexts: [B][H][P] m and l plus [B][H][P][D] partial outputs, fp32, then the
-    # fused merge's 64-bit tickets [B][Hk]
-    n = 64 * 32 * 4
-    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == (n * 128 * 4 + 2 * ((n * 4 + 15) // 16 * 16) +
-                                                             (64 * 8 * 8 + 15) // 16 * 16)
+    assert pa.pa_decode_workspace_bytes(0, 2048, 0, s) == 0
+    # one CTA (the list has 8 blocks at most)
+    assert pa.pa_decode_workspace_bytes(1, 16, 0, s) == ws_bytes(1, 1)
+    # forced: slices of about 512 tokens of a 2048-token context: 64 * 8 * 128 * 16 / 512 = 2048 slices
+    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == ws_bytes(64, 512)
     with pytest.raises(pa.PaError):
         pa.pa_decode_workspace_bytes(4, 100, 100, s)  # not a multiple of 64
 
 
-def ws_bytes(B, H, P, D=128, Hk=8):
-    n = B * H * P
-    return n * D * 4 + 2 * ((n * 4 + 15) // 16 * 16) + (B * Hk * 8 + 15) // 16 * 16
-
-
-def test_automatic_partitions():
-    # no GPU here, so the policy assumes 148 SMs: 444 resident decode CTAs at 4 query heads per KV head
+def test_automatic_slices():
+    # no GPU here, so the policy assumes 148 SMs holding 3 decode CTAs each: 444 CTAs, 1776 slices
     from paged_kv_cache_366_b200 import pa
     s = shape()
-    # 256 x 8 units fill the GPU four times over: contexts are not split
-    assert pa.pa_decode_workspace_bytes(256, 2016, 0, s) == 0
-    # 64 x 8 units: 512-token partitions (4 of them for 2048 tokens)
-    assert pa.pa_decode_workspace_bytes(64, 2048, 0, s) == ws_bytes(64, 32, 4)
-    # 8 x 8 units of 32 K tokens: 1024-token partitions (32)
-    assert pa.pa_decode_workspace_bytes(8, 32768, 0, s) == ws_bytes(8, 32, 32)
-    # one sequence of 4096 tokens: partitions shrink to 128 so the grid covers the GPU
-    assert pa.pa_decode_workspace_bytes(1, 4096, 0, s) == ws_bytes(1, 32, 32)
+    assert pa.pa_decode_workspace_bytes(64, 2048, 0, s) == ws_bytes(64, 444)
+    assert pa.pa_decode_workspace_bytes(8, 32768, 0, s) == ws_bytes(8, 444)
+    assert pa.pa_decode_workspace_bytes(256, 2016, 0, s) == ws_bytes(256, 444)
+    # one sequence of 4096 tokens: 8 * 256 blocks at most, one slice per 4 blocks: 512 slices
+    assert pa.pa_decode_workspace_bytes(1, 4096, 0, s) == ws_bytes(1, 128)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -105,8 +108,8 @@ def test_fp8_cache_shape_validation(kw, code):
 def test_null_pointers_are_rejected_before_any_launch():
     from paged_kv_cache_366_b200 import pa
     s = shape()
-    for fn in (pa.lib.pa_decode, pa.lib.pa_decode_partitions, pa.lib.pa_decode_merge):
-        assert fn(None, None, None, None, None, 4, None, 2, 64, 1.0, 0, None, 0, ctypes.byref(s), None) == -1
+    assert pa.lib.pa_decode(None, None, None, None, None, 4, None, 2, 64, 1.0, 0, None, 0, ctypes.byref(s),
+                            None) == -1
     rc = pa.lib.pa_reshape_and_cache(None, None, None, None, None, 3, ctypes.byref(s), None)
     assert rc == -1
     assert pa.lib.pa_reshape_and_cache(None, None, None, None, None, 0, ctypes.byref(s), None) == 0

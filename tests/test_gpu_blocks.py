@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from paged_kv_cache_366_b200 import workloads as W
-from gpu_util import TOL, DevCase, max_err, oracle_written, to_dev, to_host
+from gpu_util import TOL, DevCase, max_err, oracle_written, to_dev, to_host, decode_workspace
 
 pytestmark = pytest.mark.gpu
 
@@ -56,7 +56,8 @@ def test_copy_on_write_fork_then_decode(pa):
     pa.pa_copy_blocks(d.k_cache, d.v_cache, to_dev(pairs))
     pa.pa_reshape_and_cache(to_dev(k_tok), to_dev(v_tok), d.k_cache, d.v_cache, to_dev(slots))
     out = torch.empty((2, 32, 128), dtype=torch.bfloat16, device="cuda")
-    pa.pa_decode(out, to_dev(q), d.k_cache, d.v_cache, to_dev(bt), to_dev(lens), 38, case.scale)
+    pa.pa_decode(out, to_dev(q), d.k_cache, d.v_cache, to_dev(bt), to_dev(lens), 38, case.scale, 0,
+                 decode_workspace(pa, 2, 38, d.k_cache, 32))
     assert pa.pa_get_status() == 0
 
     kc, vc = oracle.copy_blocks(case.k_cache, case.v_cache, pairs)
