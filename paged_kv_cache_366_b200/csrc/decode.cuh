@@ -8,7 +8,7 @@
 // a running result. That is online softmax: a running max m, a running sum l
 // and an accumulator O rescaled by exp(m_old - m_new) whenever m grows.
 //
-// How it runs on B200 (two kernels, the second a programmatic dependent):
+// How it runs on B200 (one kernel):
 //  * Work is the flat list of (sequence, KV head, block) triples in that
 //    order; a (sequence, KV head) pair is a "unit". The grid is persistent
 //    (the CTAs all SMs hold at once) and each warp takes one of
@@ -20,7 +20,10 @@
 //  * A unit's part inside one slice is a "segment". A warp leaving a segment
 //    writes the unit's output itself when the whole unit lies in its slice;
 //    otherwise it writes the segment's partial (m, l, O) to the workspace.
-//    decode_merge_kernel then merges the partials of every cut unit.
+//    At the end of its slice a warp counts its cut segments in per-unit
+//    tickets in the workspace; the CTA of the last slice of a unit to be
+//    counted merges the unit's partials after its warps are done. A ticket
+//    carries a per-call stamp, so the workspace needs no initialisation.
 //  * Every query head of the KV head's group (G = H / Hk of them) reads each
 //    loaded block from shared memory, so K/V cross HBM once per KV head.
 //  * Each warp streams its blocks through an NSTAGE-deep shared-memory ring:
@@ -55,6 +58,7 @@ namespace pa {
 
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
+constexpr int kMergeList = 2 * kDecodeWarps;  // a warp's slice cuts at most two units
 
 template <typename T, int D, int G>
 struct DecodeCfg {
@@ -86,8 +90,9 @@ struct DecodeCfg {
     static constexpr int PBUF = kBlockSize * G * 8;         // per warp: [16 rows][G heads] of (p, p)
     static constexpr int OFF_BAR = RING_BYTES;              // NSTAGE mbarriers per warp
     static constexpr int OFF_P = OFF_BAR + kDecodeWarps * NSTAGE * 8;
-    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;  // the warps' slice starts
-    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16;
+    // the warps' slice starts, then the merge list: a count and (unit, first slot, slots)
+    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;
+    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16 + kMergeList * 12;
     // CTAs of this kernel one SM holds: the register budget or shared memory
     // (228 KB per SM, 1 KB of it reserved per CTA), whichever binds first.
     static constexpr int RESIDENT = (228 * 1024) / (SMEM + 1024) < MIN_BLOCKS ? (228 * 1024) / (SMEM + 1024)
@@ -160,7 +165,7 @@ struct DecodeParams {
     float *ws_o;   // [slots][G][D] partial outputs; slot = slice index + unit index
     float *ws_m;   // [slots][G]
     float *ws_l;   // [slots][G]
-    int *ws_unit;  // [B][Hk][2]: (first slice, slices) of each unit with blocks, written every call
+    unsigned long long *ws_ticket;  // [B][Hk] merge tickets: (call stamp << 32) | slices counted
     long long num_blocks;
     int num_seqs;
     int max_blocks_per_seq;
@@ -169,6 +174,7 @@ struct DecodeParams {
     int max_context_len;
     float scale_log2;  // softmax scale * log2(e) (times k_scale for an FP8 cache)
     float v_scale;     // 1, or the FP8 value scale
+    unsigned int stamp;  // nonzero, different for every host call: a ticket with another stamp counts as 0
 };
 
 // Position in the flat (sequence, KV head, block) list.
@@ -214,6 +220,60 @@ __device__ __forceinline__ int slice_of(long long f, long long N, int W) {
     return static_cast<int>(((f + 1) * W - 1) / N);
 }
 
+// Merge the partials of unit u held in slots s0 .. s0 + nseg - 1:
+//   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L.
+// Thread t takes four consecutive columns of one head (elements 4t, 4t + 4*nthreads,
+// ...), with every slot's loads of a round in flight together (up to 8 slots a round).
+template <typename T, int G, int D>
+__device__ __forceinline__ void merge_unit(const DecodeParams &prm, int u, int s0, int nseg, int tid, int nthreads) {
+    const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
+    for (int idx = 4 * tid; idx < G * D; idx += 4 * nthreads) {
+        const int g = idx / D, d = idx % D;
+        float M = -CUDART_INF_F, Lsum = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p0 = 0; p0 < nseg; p0 += 8) {
+            float mp[8], lp[8];
+            float4 op[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const bool in = p0 + i < nseg;
+                const size_t s = static_cast<size_t>(s0 + p0 + i);
+                mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
+                lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
+                op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float mc = M;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
+            if (mc == -CUDART_INF_F) continue;
+            const float a = exp2f(M - mc);  // 0 while M is still -inf
+            O.x *= a;
+            O.y *= a;
+            O.z *= a;
+            O.w *= a;
+            Lsum *= a;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (mp[i] == -CUDART_INF_F) continue;  // a slice whose blocks were all skipped
+                const float wt = exp2f(mp[i] - mc);
+                O.x += wt * op[i].x;
+                O.y += wt * op[i].y;
+                O.z += wt * op[i].z;
+                O.w += wt * op[i].w;
+                Lsum += wt * lp[i];
+            }
+            M = mc;
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        O.x *= inv;
+        O.y *= inv;
+        O.z *= inv;
+        O.w *= inv;
+        store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
+    }
+}
+
 // Tq: element type of q and out. Tc: element type of the caches (the same, or
 // FP8 E4M3 codes with bf16 q/out).
 template <typename Tq, typename Tc, int D, int G>
@@ -230,6 +290,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
 
     extern __shared__ __align__(128) unsigned char smem[];
     int *starts = reinterpret_cast<int *>(smem + C::OFF_MISC);  // per warp: b, hk, blk, c, nblk of its first block
+    int *merges = starts + kDecodeWarps * 5 + 4;                // [0]: count; then (unit, first slot, slots)
 
     // The lane's step and head order for the transpose-reduce: at the reduce
     // step whose partner differs in lane bit `off`, values i and i + h (h half
@@ -254,53 +315,43 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     }
 
     // Launched as a programmatic dependent (its launch overlaps the previous
-    // kernel, e.g. the cache write): wait for that kernel before reading any
-    // input. The merge kernel that follows may start its launch at once; it
-    // waits for this grid to finish before reading anything.
+    // kernel, e.g. the cache write): wait for that kernel before reading any input.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- prologue (the whole CTA): the total block count N, the slices, and
-    // the unit holding each warp's first block
+    // the unit holding each warp's first block, from prefix sums of Hk * blocks
+    // over the sequences, a chunk of sequences at a time in shared memory (the
+    // ring is not in use yet). With more sequences than one chunk holds, a
+    // first pass sums N.
+    constexpr int CHUNK = C::RING_BYTES / 8;
+    long long *cum = reinterpret_cast<long long *>(smem);
     long long N = 0;
-    {
+    if (threadIdx.x == 0) merges[0] = 0;
+    if (B > CHUNK) {
         long long part = 0;
         for (int b = threadIdx.x; b < B; b += kDecodeThreads) {
-            const int c = clamp_context(__ldg(prm.context_lens + b), cap, blockIdx.x == 0);
+            const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
             part += (c + kBlockSize - 1) / kBlockSize;
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        long long *red64 = reinterpret_cast<long long *>(smem);
-        if (lane == 0) red64[warp] = part;
+        if (lane == 0) cum[warp] = part;
         __syncthreads();
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) N += red64[w];
+        for (int w = 0; w < kDecodeWarps; ++w) N += cum[w];
         N *= Hk;
         __syncthreads();
     }
-    // Sequences of length 0 have no blocks: CTA b % gridDim.x writes their zero rows.
-    for (int b = blockIdx.x; b < B; b += gridDim.x) {
-        if (clamp_context(__ldg(prm.context_lens + b), cap, false) != 0) continue;
-        Tq *o = static_cast<Tq *>(prm.out) + static_cast<size_t>(b) * prm.num_heads * D;
-        for (int i = threadIdx.x; i < prm.num_heads * D; i += kDecodeThreads) store_out(o + i, 0.f);
-    }
-    // WS slices, at most one per block, so that none is empty (a unit's slices
-    // are then exactly those from the slice of its first block to that of its last)
-    const int WS = static_cast<int>(min(static_cast<long long>(gridDim.x) * kDecodeWarps, N));
     const int cta0 = static_cast<int>(blockIdx.x) * kDecodeWarps;  // first slice of this CTA
-    if (cta0 >= WS) return;
+    int WS = 0;  // slices: at most one per block, so that none is empty (a unit's slices are then
+                 // exactly those from the slice of its first block to that of its last)
     {
-        // Locate each warp's first block: prefix sums of Hk * blocks over the
-        // sequences, a chunk of sequences at a time in shared memory (the ring
-        // is not in use yet).
-        constexpr int CHUNK = C::RING_BYTES / 8;
-        long long *cum = reinterpret_cast<long long *>(smem);
         long long base = 0;
         for (int c0 = 0; c0 < B; c0 += CHUNK) {
             const int n = min(CHUNK, B - c0);
             for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
-                const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
+                const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, blockIdx.x == 0);
                 cum[i] = static_cast<long long>((c + kBlockSize - 1) / kBlockSize) * Hk;
             }
             __syncthreads();
@@ -319,20 +370,29 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
                 }
             }
             __syncthreads();
+            if (B <= CHUNK) N = cum[n - 1];  // one chunk: the total comes with the scan
+            WS = static_cast<int>(min(static_cast<long long>(gridDim.x) * kDecodeWarps, N));
             for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
                 const long long hi = cum[i], lo = i ? cum[i - 1] : base;
-                if (lo >= hi) continue;
+                if (lo >= hi) {
+                    // a sequence of length 0 has no blocks: CTA b % gridDim.x writes its zero rows
+                    const int b = c0 + i;
+                    if (b % static_cast<int>(gridDim.x) == static_cast<int>(blockIdx.x)) {
+                        Tq *o = static_cast<Tq *>(prm.out) + static_cast<size_t>(b) * prm.num_heads * D;
+                        for (int e = 0; e < prm.num_heads * D; ++e) store_out(o + e, 0.f);
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int w = 0; w < kDecodeWarps; ++w) {
-                    const long long f = N * (cta0 + w) / WS;  // first block of slice cta0 + w
-                    if (cta0 + w < WS && lo <= f && f < hi) {  // ... lies in sequence c0 + i
-                        const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
-                        const int nblk = (c + kBlockSize - 1) / kBlockSize;
+                    const long long f = N * (cta0 + w) / max(WS, 1);  // first block of slice cta0 + w
+                    if (cta0 + w < WS && lo <= f && f < hi) {         // ... lies in sequence c0 + i
+                        const int nblk = static_cast<int>((hi - lo) / Hk);
                         const long long r = f - lo;
                         starts[5 * w + 0] = c0 + i;
                         starts[5 * w + 1] = static_cast<int>(r / nblk);
                         starts[5 * w + 2] = static_cast<int>(r % nblk);
-                        starts[5 * w + 3] = c;
+                        starts[5 * w + 3] = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
                         starts[5 * w + 4] = nblk;
                     }
                 }
@@ -341,10 +401,10 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             __syncthreads();
         }
     }
-    // ---- from here on every warp runs alone on its slice
+    if (cta0 >= WS) return;
+    // ---- from here on every warp runs alone on its slice, until the merges
     const int slice = cta0 + warp;
-    if (slice >= WS) return;
-    const long long s_lo = N * slice / WS, s_hi = N * (slice + 1) / WS;
+    const long long s_lo = slice < WS ? N * slice / WS : 0, s_hi = slice < WS ? N * (slice + 1) / WS : 0;
     const int nb_w = static_cast<int>(s_hi - s_lo);
 
     unsigned char *ring = smem + warp * C::WARP_RING;
@@ -358,8 +418,12 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         fence_mbar_init();
     }
     __syncwarp();
-    Cursor cc{0, starts[5 * warp], starts[5 * warp + 1], starts[5 * warp + 3], starts[5 * warp + 4],
-              starts[5 * warp + 2]};
+    Cursor cc{0, 0, 0, 0, 1, 0};
+    if (nb_w > 0)
+        cc = Cursor{0, starts[5 * warp], starts[5 * warp + 1], starts[5 * warp + 3], starts[5 * warp + 4],
+                    starts[5 * warp + 2]};
+    // this slice's cut units (at most its first and its last): unit, first slice, slices
+    int cut_u0 = 0, cut_c0 = 0, cut_n0 = 0, cut_u1 = 0, cut_c1 = 0, cut_n1 = 0, ncut = 0;
 
     // ---- issue side: block k of this warp at cursor ic (NSTAGE blocks ahead of
     // the block being consumed), with the next 32 table entries of its unit
@@ -519,10 +583,18 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             prm.ws_m[slot * G + lane] = m;
             prm.ws_l[slot * G + lane] = l;
         }
-        if (lane == 0 && u_lo >= s_lo) {  // the unit starts in this slice: where its partials are
-            int *rec = prm.ws_unit + 2 * static_cast<size_t>(u);
-            rec[0] = slice;
-            rec[1] = whole ? 1 : slice_of(u_hi - 1, N, WS) - slice + 1;
+        if (!whole && ncut < 2) {  // only the first and the last segment of a slice can be cut
+            const int c1 = slice_of(u_lo, N, WS), n = slice_of(u_hi - 1, N, WS) - c1 + 1;
+            if (ncut == 0) {
+                cut_u0 = u;
+                cut_c0 = c1;
+                cut_n0 = n;
+            } else {
+                cut_u1 = u;
+                cut_c1 = c1;
+                cut_n1 = n;
+            }
+            ++ncut;
         }
     };
 
@@ -694,70 +766,42 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         // flight land before the CTA ends.
         for (int kk = k; kk < min(k + C::NSTAGE, nb_w); ++kk)
             mbar_wait(bars + 8 * (kk % C::NSTAGE), (kk / C::NSTAGE) & 1);
+        ncut = 0;
     }
-}
 
-// Merge the partials of every unit cut by slice boundaries:
-//   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L
-// over the unit's slices s (slots first + u .. first + slices - 1 + u). Grid
-// (units, G*D/128 column groups); a thread takes four consecutive columns of one
-// head, with every slot's loads of a round in flight together (up to 8 slots a
-// round). A programmatic dependent of decode_kernel: it waits for it before
-// reading the workspace.
-template <typename T, int G, int D>
-__global__ void __launch_bounds__(32) decode_merge_kernel(const DecodeParams prm) {
-    const int u = blockIdx.x;
-    const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
-    const int idx = 4 * (blockIdx.y * 32 + threadIdx.x);
-    if (idx >= G * D) return;
-    if (clamp_context(__ldg(prm.context_lens + b), decode_cap(prm), false) == 0) return;  // zero rows, written
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int first = __ldcg(prm.ws_unit + 2 * u), nseg = __ldcg(prm.ws_unit + 2 * u + 1);
-    if (nseg <= 1) return;  // a whole unit: written by the decode kernel
-    const int g = idx / D, d = idx % D;
-    const int s0 = first + u;
-    float M = -CUDART_INF_F, Lsum = 0.f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = 0; p0 < nseg; p0 += 8) {
-        float mp[8], lp[8];
-        float4 op[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const bool in = p0 + i < nseg;
-            const size_t s = static_cast<size_t>(s0 + p0 + i);
-            mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
-            lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
-            op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    // ---- count this slice's cut segments in their units' tickets; the last
+    // slice of a unit to be counted has its CTA merge the unit's partials
+    __syncwarp();  // the lanes' partial writes, before lane 0's fence
+    if (lane == 0 && ncut > 0) {
+        __threadfence();  // the partials, before the tickets
+        const unsigned long long stamp = static_cast<unsigned long long>(prm.stamp) << 32;
+        for (int i = 0; i < ncut; ++i) {
+            const int cu = i ? cut_u1 : cut_u0, cc1 = i ? cut_c1 : cut_c0, cn = i ? cut_n1 : cut_n0;
+            unsigned long long *ticket = prm.ws_ticket + cu;
+            unsigned long long cur = __ldcg(ticket), seen;
+            unsigned int n;
+            do {
+                seen = cur;
+                n = (seen & 0xffffffff00000000ull) == stamp ? static_cast<unsigned int>(seen) : 0u;
+                cur = atomicCAS(ticket, seen, stamp | (n + 1u));
+            } while (cur != seen);
+            if (n + 1u == static_cast<unsigned int>(cn)) {
+                const int at = atomicAdd(merges, 1);
+                merges[1 + 3 * at] = cu;
+                merges[2 + 3 * at] = cc1 + cu;
+                merges[3 + 3 * at] = cn;
+            }
         }
-        float mc = M;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
-        if (mc == -CUDART_INF_F) continue;
-        const float a = exp2f(M - mc);  // 0 while M is still -inf
-        O.x *= a;
-        O.y *= a;
-        O.z *= a;
-        O.w *= a;
-        Lsum *= a;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (mp[i] == -CUDART_INF_F) continue;  // a slice whose blocks were all skipped
-            const float wt = exp2f(mp[i] - mc);
-            O.x += wt * op[i].x;
-            O.y += wt * op[i].y;
-            O.z += wt * op[i].z;
-            O.w += wt * op[i].w;
-            Lsum += wt * lp[i];
-        }
-        M = mc;
     }
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    O.x *= inv;
-    O.y *= inv;
-    O.z *= inv;
-    O.w *= inv;
-    store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
+    __syncthreads();
+    const int nm = merges[0];
+    if (nm == 0) return;
+    __threadfence();  // every other slice's partials, after their tickets
+    for (int i = 0; i < nm; ++i)
+        merge_unit<Tq, G, D>(prm, merges[1 + 3 * i], merges[2 + 3 * i], merges[3 + 3 * i], threadIdx.x,
+                             kDecodeThreads);
+    if (threadIdx.x < nm)  // no slice counted: a replay of this launch starts afresh
+        atomicExch(prm.ws_ticket + merges[1 + 3 * threadIdx.x], static_cast<unsigned long long>(prm.stamp) << 32);
 }
 
 }  // namespace pa
