@@ -132,7 +132,8 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
  * when num_seqs is 0. Negative on bad arguments.
  * With S slices (see pa_decode) and U = B * Hk units the layout is: fp32
  * partial outputs [S + U - 1][G][D], partial maxima and sums [S + U - 1][G]
- * each, then 64-bit merge tickets [U], each part 16-byte aligned (G = H / Hk).
+ * each, then int32 (first slice, slices) records [U], each part 16-byte
+ * aligned (G = H / Hk).
  */
 int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int32_t partition_tokens,
                                   const pa_shape *shape);
@@ -159,8 +160,7 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
  *                  16-token block) items is cut into S equal slices, one per
  *                  warp of a persistent grid; a (sequence, KV head) cut by
  *                  slice boundaries gets one partial (max, sum, unnormalised
- *                  O) per slice in the workspace, and the CTA of the last of
- *                  its slices to finish (a ticket in the workspace) merges
+ *                  O) per slice in the workspace, and a second kernel merges
  *                  them. Automatic S: the warps of all the decode CTAs the SMs
  *                  hold at once, at most one per 4 blocks of
  *                  B * Hk * ceil(max_context_len / 16). Otherwise a multiple
@@ -169,14 +169,11 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
  *                  more, smaller slices).
  *   workspace    : device scratch of >= pa_decode_workspace_bytes(...) bytes,
  *                  16-byte aligned. Its contents need no initialisation: a
- *                  call writes every partial before it reads it, and each
- *                  ticket holds a stamp of the call that wrote it (different
- *                  for every host call, kept by a CUDA graph replay, which
- *                  leaves its tickets reset); a ticket with another stamp
- *                  counts as empty. Calls that overlap on the GPU must not
- *                  share a workspace.
+ *                  call writes every partial and record before it reads it.
+ *                  Calls that overlap on the GPU must not share a workspace.
  * Accumulation is fp32 whatever the dtype. bf16 output is rounded once, to
- * nearest even. One kernel launch.
+ * nearest even. Two kernel launches, the second a programmatic dependent of
+ * the first.
  */
 int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
               int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
@@ -273,11 +270,10 @@ int pa_swap_blocks(void *dst, const void *src, const int64_t *block_pairs, int64
  *    Use pa_decode with your own workspace for those, or a larger
  *    partition_tokens.
  *  - Every call on a device shares the one array, and the array keeps whatever
- *    the last call left in it. A call first zeroes the merge tickets it will
- *    use (an asynchronous memset on `stream`) and writes every partial before
- *    it reads it, so no earlier call's contents matter. Calls that may overlap
- *    on the GPU (different streams, or different host threads on one device)
- *    race on the array and must be serialized by the caller.
+ *    the last call left in it. Nothing in it needs to start at zero: a call
+ *    writes every partial and record before it reads it. Calls that may
+ *    overlap on the GPU (different streams, or different host threads on one
+ *    device) race on the array and must be serialized by the caller.
  * The library calls no cudaMalloc, cudaFree or other allocating routine here.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -8,7 +8,7 @@
 // a running result. That is online softmax: a running max m, a running sum l
 // and an accumulator O rescaled by exp(m_old - m_new) whenever m grows.
 //
-// How it runs on B200 (one kernel):
+// How it runs on B200 (two kernels, the second a programmatic dependent):
 //  * Work is the flat list of (sequence, KV head, block) triples in that
 //    order; a (sequence, KV head) pair is a "unit". The grid is persistent
 //    (the CTAs all SMs hold at once) and each warp takes one of
@@ -20,10 +20,7 @@
 //  * A unit's part inside one slice is a "segment". A warp leaving a segment
 //    writes the unit's output itself when the whole unit lies in its slice;
 //    otherwise it writes the segment's partial (m, l, O) to the workspace.
-//    At the end of its slice a warp counts its cut segments in per-unit
-//    tickets in the workspace; the CTA of the last slice of a unit to be
-//    counted merges the unit's partials after its warps are done. A ticket
-//    carries a per-call stamp, so the workspace needs no initialisation.
+//    decode_merge_kernel then merges the partials of every cut unit.
 //  * Every query head of the KV head's group (G = H / Hk of them) reads each
 //    loaded block from shared memory, so K/V cross HBM once per KV head.
 //  * Each warp streams its blocks through an NSTAGE-deep shared-memory ring:
@@ -58,7 +55,6 @@ namespace pa {
 
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
-constexpr int kMergeList = 2 * kDecodeWarps;  // a warp's slice cuts at most two units
 
 template <typename T, int D, int G>
 struct DecodeCfg {
@@ -90,9 +86,8 @@ struct DecodeCfg {
     static constexpr int PBUF = kBlockSize * G * 8;         // per warp: [16 rows][G heads] of (p, p)
     static constexpr int OFF_BAR = RING_BYTES;              // NSTAGE mbarriers per warp
     static constexpr int OFF_P = OFF_BAR + kDecodeWarps * NSTAGE * 8;
-    // the warps' slice starts, then the merge list: a count and (unit, first slot, slots)
-    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;
-    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16 + kMergeList * 12;
+    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;  // the warps' slice starts
+    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16;
     // CTAs of this kernel one SM holds: the register budget or shared memory
     // (228 KB per SM, 1 KB of it reserved per CTA), whichever binds first.
     static constexpr int RESIDENT = (228 * 1024) / (SMEM + 1024) < MIN_BLOCKS ? (228 * 1024) / (SMEM + 1024)
@@ -165,7 +160,7 @@ struct DecodeParams {
     float *ws_o;   // [slots][G][D] partial outputs; slot = slice index + unit index
     float *ws_m;   // [slots][G]
     float *ws_l;   // [slots][G]
-    unsigned long long *ws_ticket;  // [B][Hk] merge tickets: (call stamp << 32) | slices counted
+    int *ws_unit;  // [B][Hk][2]: (first slice, slices) of each unit with blocks, written every call
     long long num_blocks;
     int num_seqs;
     int max_blocks_per_seq;
@@ -174,7 +169,6 @@ struct DecodeParams {
     int max_context_len;
     float scale_log2;  // softmax scale * log2(e) (times k_scale for an FP8 cache)
     float v_scale;     // 1, or the FP8 value scale
-    unsigned int stamp;  // nonzero, different for every host call: a ticket with another stamp counts as 0
 };
 
 // Position in the flat (sequence, KV head, block) list.
@@ -220,60 +214,6 @@ __device__ __forceinline__ int slice_of(long long f, long long N, int W) {
     return static_cast<int>(((f + 1) * W - 1) / N);
 }
 
-// Merge the partials of unit u held in slots s0 .. s0 + nseg - 1:
-//   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L.
-// Thread t takes four consecutive columns of one head (elements 4t, 4t + 4*nthreads,
-// ...), with every slot's loads of a round in flight together (up to 8 slots a round).
-template <typename T, int G, int D>
-__device__ __forceinline__ void merge_unit(const DecodeParams &prm, int u, int s0, int nseg, int tid, int nthreads) {
-    const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
-    for (int idx = 4 * tid; idx < G * D; idx += 4 * nthreads) {
-        const int g = idx / D, d = idx % D;
-        float M = -CUDART_INF_F, Lsum = 0.f;
-        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p0 = 0; p0 < nseg; p0 += 8) {
-            float mp[8], lp[8];
-            float4 op[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const bool in = p0 + i < nseg;
-                const size_t s = static_cast<size_t>(s0 + p0 + i);
-                mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
-                lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
-                op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            float mc = M;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
-            if (mc == -CUDART_INF_F) continue;
-            const float a = exp2f(M - mc);  // 0 while M is still -inf
-            O.x *= a;
-            O.y *= a;
-            O.z *= a;
-            O.w *= a;
-            Lsum *= a;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (mp[i] == -CUDART_INF_F) continue;  // a slice whose blocks were all skipped
-                const float wt = exp2f(mp[i] - mc);
-                O.x += wt * op[i].x;
-                O.y += wt * op[i].y;
-                O.z += wt * op[i].z;
-                O.w += wt * op[i].w;
-                Lsum += wt * lp[i];
-            }
-            M = mc;
-        }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        O.x *= inv;
-        O.y *= inv;
-        O.z *= inv;
-        O.w *= inv;
-        store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
-    }
-}
-
 // Tq: element type of q and out. Tc: element type of the caches (the same, or
 // FP8 E4M3 codes with bf16 q/out).
 template <typename Tq, typename Tc, int D, int G>
@@ -290,7 +230,6 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
 
     extern __shared__ __align__(128) unsigned char smem[];
     int *starts = reinterpret_cast<int *>(smem + C::OFF_MISC);  // per warp: b, hk, blk, c, nblk of its first block
-    int *merges = starts + kDecodeWarps * 5 + 4;                // [0]: count; then (unit, first slot, slots)
 
     // The lane's step and head order for the transpose-reduce: at the reduce
     // step whose partner differs in lane bit `off`, values i and i + h (h half
@@ -315,7 +254,9 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     }
 
     // Launched as a programmatic dependent (its launch overlaps the previous
-    // kernel, e.g. the cache write): wait for that kernel before reading any input.
+    // kernel, e.g. the cache write): wait for that kernel before reading any
+    // input. The merge kernel that follows may start its launch at once; it
+    // waits for this grid to finish before reading anything.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -327,7 +268,6 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     constexpr int CHUNK = C::RING_BYTES / 8;
     long long *cum = reinterpret_cast<long long *>(smem);
     long long N = 0;
-    if (threadIdx.x == 0) merges[0] = 0;
     if (B > CHUNK) {
         long long part = 0;
         for (int b = threadIdx.x; b < B; b += kDecodeThreads) {
@@ -402,9 +342,10 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         }
     }
     if (cta0 >= WS) return;
-    // ---- from here on every warp runs alone on its slice, until the merges
+    // ---- from here on every warp runs alone on its slice
     const int slice = cta0 + warp;
-    const long long s_lo = slice < WS ? N * slice / WS : 0, s_hi = slice < WS ? N * (slice + 1) / WS : 0;
+    if (slice >= WS) return;
+    const long long s_lo = N * slice / WS, s_hi = N * (slice + 1) / WS;
     const int nb_w = static_cast<int>(s_hi - s_lo);
 
     unsigned char *ring = smem + warp * C::WARP_RING;
@@ -418,12 +359,8 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         fence_mbar_init();
     }
     __syncwarp();
-    Cursor cc{0, 0, 0, 0, 1, 0};
-    if (nb_w > 0)
-        cc = Cursor{0, starts[5 * warp], starts[5 * warp + 1], starts[5 * warp + 3], starts[5 * warp + 4],
-                    starts[5 * warp + 2]};
-    // this slice's cut units (at most its first and its last): unit, first slice, slices
-    int cut_u0 = 0, cut_c0 = 0, cut_n0 = 0, cut_u1 = 0, cut_c1 = 0, cut_n1 = 0, ncut = 0;
+    Cursor cc{0, starts[5 * warp], starts[5 * warp + 1], starts[5 * warp + 3], starts[5 * warp + 4],
+              starts[5 * warp + 2]};
 
     // ---- issue side: block k of this warp at cursor ic (NSTAGE blocks ahead of
     // the block being consumed), with the next 32 table entries of its unit
@@ -583,18 +520,10 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             prm.ws_m[slot * G + lane] = m;
             prm.ws_l[slot * G + lane] = l;
         }
-        if (!whole && ncut < 2) {  // only the first and the last segment of a slice can be cut
-            const int c1 = slice_of(u_lo, N, WS), n = slice_of(u_hi - 1, N, WS) - c1 + 1;
-            if (ncut == 0) {
-                cut_u0 = u;
-                cut_c0 = c1;
-                cut_n0 = n;
-            } else {
-                cut_u1 = u;
-                cut_c1 = c1;
-                cut_n1 = n;
-            }
-            ++ncut;
+        if (lane == 0 && u_lo >= s_lo) {  // the unit starts in this slice: where its partials are
+            int *rec = prm.ws_unit + 2 * static_cast<size_t>(u);
+            rec[0] = slice;
+            rec[1] = whole ? 1 : slice_of(u_hi - 1, N, WS) - slice + 1;
         }
     };
 
@@ -766,42 +695,70 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         // flight land before the CTA ends.
         for (int kk = k; kk < min(k + C::NSTAGE, nb_w); ++kk)
             mbar_wait(bars + 8 * (kk % C::NSTAGE), (kk / C::NSTAGE) & 1);
-        ncut = 0;
     }
+}
 
-    // ---- count this slice's cut segments in their units' tickets; the last
-    // slice of a unit to be counted has its CTA merge the unit's partials
-    __syncwarp();  // the lanes' partial writes, before lane 0's fence
-    if (lane == 0 && ncut > 0) {
-        __threadfence();  // the partials, before the tickets
-        const unsigned long long stamp = static_cast<unsigned long long>(prm.stamp) << 32;
-        for (int i = 0; i < ncut; ++i) {
-            const int cu = i ? cut_u1 : cut_u0, cc1 = i ? cut_c1 : cut_c0, cn = i ? cut_n1 : cut_n0;
-            unsigned long long *ticket = prm.ws_ticket + cu;
-            unsigned long long cur = __ldcg(ticket), seen;
-            unsigned int n;
-            do {
-                seen = cur;
-                n = (seen & 0xffffffff00000000ull) == stamp ? static_cast<unsigned int>(seen) : 0u;
-                cur = atomicCAS(ticket, seen, stamp | (n + 1u));
-            } while (cur != seen);
-            if (n + 1u == static_cast<unsigned int>(cn)) {
-                const int at = atomicAdd(merges, 1);
-                merges[1 + 3 * at] = cu;
-                merges[2 + 3 * at] = cc1 + cu;
-                merges[3 + 3 * at] = cn;
-            }
+// Merge the partials of every unit cut by slice boundaries:
+//   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L
+// over the unit's slices s (slots first + u .. first + slices - 1 + u). Grid
+// (units, G*D/128 column groups); a thread takes four consecutive columns of one
+// head, with every slot's loads of a round in flight together (up to 8 slots a
+// round). A programmatic dependent of decode_kernel: it waits for it before
+// reading the workspace.
+template <typename T, int G, int D>
+__global__ void __launch_bounds__(32) decode_merge_kernel(const DecodeParams prm) {
+    const int u = blockIdx.x;
+    const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
+    const int idx = 4 * (blockIdx.y * 32 + threadIdx.x);
+    if (idx >= G * D) return;
+    if (clamp_context(__ldg(prm.context_lens + b), decode_cap(prm), false) == 0) return;  // zero rows, written
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int first = __ldcg(prm.ws_unit + 2 * u), nseg = __ldcg(prm.ws_unit + 2 * u + 1);
+    if (nseg <= 1) return;  // a whole unit: written by the decode kernel
+    const int g = idx / D, d = idx % D;
+    const int s0 = first + u;
+    float M = -CUDART_INF_F, Lsum = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < nseg; p0 += 8) {
+        float mp[8], lp[8];
+        float4 op[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool in = p0 + i < nseg;
+            const size_t s = static_cast<size_t>(s0 + p0 + i);
+            mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
+            lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
+            op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        float mc = M;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mc = fmaxf(mc, mp[i]);
+        if (mc == -CUDART_INF_F) continue;
+        const float a = exp2f(M - mc);  // 0 while M is still -inf
+        O.x *= a;
+        O.y *= a;
+        O.z *= a;
+        O.w *= a;
+        Lsum *= a;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (mp[i] == -CUDART_INF_F) continue;  // a slice whose blocks were all skipped
+            const float wt = exp2f(mp[i] - mc);
+            O.x += wt * op[i].x;
+            O.y += wt * op[i].y;
+            O.z += wt * op[i].z;
+            O.w += wt * op[i].w;
+            Lsum += wt * lp[i];
+        }
+        M = mc;
     }
-    __syncthreads();
-    const int nm = merges[0];
-    if (nm == 0) return;
-    __threadfence();  // every other slice's partials, after their tickets
-    for (int i = 0; i < nm; ++i)
-        merge_unit<Tq, G, D>(prm, merges[1 + 3 * i], merges[2 + 3 * i], merges[3 + 3 * i], threadIdx.x,
-                             kDecodeThreads);
-    if (threadIdx.x < nm)  // no slice counted: a replay of this launch starts afresh
-        atomicExch(prm.ws_ticket + merges[1 + 3 * threadIdx.x], static_cast<unsigned long long>(prm.stamp) << 32);
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    O.x *= inv;
+    O.y *= inv;
+    O.z *= inv;
+    O.w *= inv;
+    store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
 }
 
 }  // namespace pa

@@ -130,8 +130,8 @@ int64_t round16(int64_t n) { return (n + 15) / 16 * 16; }
 // waves), but no more than one warp per 4 blocks of the largest possible list.
 // With partition_tokens given: slices of about that many tokens of a context
 // of max_context_len. Workspace: fp32 partial outputs [slots][G][D], partial
-// maxima and sums [slots][G] each, then 64-bit merge tickets [B][Hk]; each
-// part 16-byte aligned.
+// maxima and sums [slots][G] each, then int32 (first slice, slices) records
+// [B][Hk]; each part 16-byte aligned.
 int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested, const pa_shape *s,
                     DecodeGeometry *g) {
     if (num_seqs < 0 || max_context_len < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -159,19 +159,6 @@ int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested
     return PA_OK;
 }
 
-// A stamp per launch for the merge tickets: nonzero (a zeroed workspace holds
-// stamp 0) and different from the stamps of recent launches. A launch captured
-// in a CUDA graph keeps its stamp on every replay; the CTAs that merge put
-// their units' tickets back to (stamp, 0), so replays start afresh too.
-uint32_t next_stamp() {
-    static std::atomic<uint32_t> counter{0};
-    uint32_t s;
-    do {
-        s = counter.fetch_add(1, std::memory_order_relaxed) + 1;
-    } while (s == 0);
-    return s;
-}
-
 template <typename Tq, typename Tc, int D, int G>
 int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaStream_t st) {
     using C = pa::DecodeCfg<Tc, D, G>;
@@ -183,8 +170,9 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaSt
         !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
         return PA_ERR_UNSUPPORTED;
-    // A programmatic dependent launch: it starts launching while the kernel
-    // before it drains, and waits for it (griddepcontrol.wait) before reading.
+    // Both kernels are programmatic dependent launches: each starts launching
+    // while the kernel before it drains, and waits for it (griddepcontrol.wait)
+    // before reading what it wrote.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -195,9 +183,12 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaSt
     cfg.gridDim = dim3(geo.ctas);
     cfg.blockDim = dim3(pa::kDecodeThreads);
     cfg.dynamicSmemBytes = C::SMEM;
-    pa::DecodeParams p = prm;
-    p.stamp = next_stamp();
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, p, tm_k, tm_v);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cfg.gridDim = dim3(static_cast<unsigned>(prm.num_seqs) * prm.num_kv_heads, (G * D + 127) / 128);
+    cfg.blockDim = dim3(32);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D>, prm);
     return e == cudaSuccess ? PA_OK : cuda_fail(e);
 }
 
@@ -279,12 +270,11 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
 
 namespace {
 
-// pa_decode after its argument checks; ticket_clear also zeroes the merge
-// tickets first (pa_decode_noalloc's shared scratch).
+// pa_decode after its argument checks.
 int decode_call(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                 int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
                 float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
-                const pa_shape *shape, void *stream, bool ticket_clear) {
+                const pa_shape *shape, void *stream) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -309,12 +299,7 @@ int decode_call(void *out, const void *q, const void *k_cache, const void *v_cac
         prm.ws_o = reinterpret_cast<float *>(w);
         prm.ws_m = reinterpret_cast<float *>(w + o_bytes);
         prm.ws_l = reinterpret_cast<float *>(w + o_bytes + ml_bytes);
-        prm.ws_ticket = reinterpret_cast<unsigned long long *>(w + o_bytes + 2 * ml_bytes);
-        if (ticket_clear) {
-            const cudaError_t e =
-                cudaMemsetAsync(prm.ws_ticket, 0, static_cast<size_t>(num_seqs) * shape->num_kv_heads * 8, st);
-            if (e != cudaSuccess) return cuda_fail(e);
-        }
+        prm.ws_unit = reinterpret_cast<int *>(w + o_bytes + 2 * ml_bytes);
     }
     prm.out = out;
     prm.q = q;
@@ -356,7 +341,7 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes, const pa_shape *shape,
               void *stream) {
     return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                       max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream, false);
+                       max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -456,10 +441,10 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
     }
     if (need == 0) return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                                     num_seqs, max_context_len, scale, partition_tokens, nullptr, 0, shape, stream);
-    // The tickets are the only part of the scratch a call reads before writing
-    // it; they are cleared first, so no earlier call's contents matter.
+    // Every partial and record a call reads, it has written first: no earlier
+    // call's contents matter.
     return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                       max_context_len, scale, partition_tokens, scratch, need, shape, stream, true);
+                       max_context_len, scale, partition_tokens, scratch, need, shape, stream);
 }
 
 static int launch_copy(void *dst, const void *src, const int64_t *pairs, int64_t num_pairs, int64_t src_blocks,
