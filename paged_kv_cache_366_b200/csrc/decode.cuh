@@ -53,8 +53,8 @@
 
 namespace pa {
 
-constexpr int kDecodeWarps = 4;
-constexpr int kDecodeThreads = 32 * kDecodeWarps;
+// Dynamic shared memory one CTA may use on sm_100.
+constexpr int kCtaSmem = 227 * 1024;
 
 template <typename T, int D, int G>
 struct DecodeCfg {
@@ -76,29 +76,39 @@ struct DecodeCfg {
     // Two stages per warp and three CTAs per SM (12 warps) measured faster on
     // B200 than three stages at two CTAs per SM.
     static constexpr int NSTAGE = 2;
-    // CTAs per SM the register budget is sized for (wide rows keep more live state).
-    static constexpr int MIN_BLOCKS = G <= 4 ? 3 : 2;
     static constexpr int WARP_RING = NSTAGE * STAGE_BYTES;
-    static constexpr int RING_BYTES = kDecodeWarps * WARP_RING;
     static constexpr int NPART = STEPS * G;                 // q.k partials per lane per block
     static constexpr int NFIN = NPART >= L ? NPART / L : 1; // complete scores per lane
     static constexpr int DUP = NPART >= L ? 1 : L / NPART;  // lanes holding the same scores
     static constexpr int PBUF = kBlockSize * G * 8;         // per warp: [16 rows][G heads] of (p, p)
-    static constexpr int OFF_BAR = RING_BYTES;              // NSTAGE mbarriers per warp
-    static constexpr int OFF_P = OFF_BAR + kDecodeWarps * NSTAGE * 8;
-    static constexpr int OFF_MISC = OFF_P + kDecodeWarps * PBUF;  // the warps' slice starts
-    static constexpr int SMEM = OFF_MISC + kDecodeWarps * 5 * 4 + 16;
-    // CTAs of this kernel one SM holds: the register budget or shared memory
-    // (228 KB per SM, 1 KB of it reserved per CTA), whichever binds first.
-    static constexpr int RESIDENT = (228 * 1024) / (SMEM + 1024) < MIN_BLOCKS ? (228 * 1024) / (SMEM + 1024)
-                                                                              : MIN_BLOCKS;
+    // One unit's queries (bf16 with an FP8 cache), fetched with the first block
+    // of each segment into that block's stage.
+    static constexpr int QBYTES = G * D * (E == 1 ? 2 : E);
+    static constexpr int WARP_Q = NSTAGE * QBYTES;
+    // Warps of one CTA, the CTA filling its SM: 12 (8 for wide groups, whose
+    // live state takes more registers), or fewer where their rings would not
+    // fit in shared memory (fp32 rows of 128). One CTA of 12 warps measured
+    // faster on B200 than three CTAs of 4 with the same rings.
+    static constexpr int WARPS_REG = G <= 4 ? 12 : 8;
+    static constexpr int WARPS_SMEM = (kCtaSmem - 1024) / (WARP_RING + WARP_Q + PBUF + NSTAGE * 8 + 20);
+    static constexpr int WARPS = WARPS_REG < WARPS_SMEM ? WARPS_REG : WARPS_SMEM;
+    static constexpr int THREADS = 32 * WARPS;
+    static constexpr int RING_BYTES = WARPS * WARP_RING;
+    static constexpr int OFF_Q = RING_BYTES;                // NSTAGE query slots per warp
+    static constexpr int OFF_BAR = OFF_Q + WARPS * WARP_Q;  // NSTAGE mbarriers per warp
+    static constexpr int OFF_P = OFF_BAR + WARPS * NSTAGE * 8;
+    static constexpr int OFF_MISC = OFF_P + WARPS * PBUF;   // the warps' slice starts
+    static constexpr int SMEM = OFF_MISC + WARPS * 5 * 4 + 16;
+    // CTAs of this kernel one SM holds, without a device to ask.
+    static constexpr int RESIDENT = 1;
     static_assert(R % (CB * CH) == 0 && L >= 1 && L <= 32 && 32 % L == 0, "row must split into lane slices");
     static_assert(kBlockSize % RS == 0, "rows per step must divide the block");
     static_assert(32 % G == 0 && G <= 8, "group size");
     static_assert(G % NFIN == 0, "a lane's scores are consecutive heads of one row");
-    static_assert(OFF_P % 16 == 0 && OFF_MISC % 16 == 0, "shared-memory alignment");
+    static_assert(OFF_P % 16 == 0 && OFF_MISC % 16 == 0 && QBYTES % 16 == 0, "shared-memory alignment");
     static_assert(STEPS >= 2 && L >= 4, "the first reduce step pairs step slots s and s + STEPS / 2");
-    static_assert(RESIDENT >= 1, "one CTA must fit an SM");
+    static_assert(SMEM <= kCtaSmem && WARPS >= 1, "one CTA must fit an SM");
+    static_assert(NSTAGE == 2, "the fetch of block k + 2 learns from one step whether it starts a unit");
 };
 
 // Sum, over the lanes that differ in the bits OFF, OFF/2, ..., 1, the N values
@@ -217,7 +227,7 @@ __device__ __forceinline__ int slice_of(long long f, long long N, int W) {
 // Tq: element type of q and out. Tc: element type of the caches (the same, or
 // FP8 E4M3 codes with bf16 q/out).
 template <typename Tq, typename Tc, int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCKS)
+__global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
     decode_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
     using C = DecodeCfg<Tc, D, G>;
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     long long N = 0;
     if (B > CHUNK) {
         long long part = 0;
-        for (int b = threadIdx.x; b < B; b += kDecodeThreads) {
+        for (int b = threadIdx.x; b < B; b += C::THREADS) {
             const int c = clamp_context(__ldg(prm.context_lens + b), cap, false);
             part += (c + kBlockSize - 1) / kBlockSize;
         }
@@ -279,18 +289,18 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         if (lane == 0) cum[warp] = part;
         __syncthreads();
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) N += cum[w];
+        for (int w = 0; w < C::WARPS; ++w) N += cum[w];
         N *= Hk;
         __syncthreads();
     }
-    const int cta0 = static_cast<int>(blockIdx.x) * kDecodeWarps;  // first slice of this CTA
+    const int cta0 = static_cast<int>(blockIdx.x) * C::WARPS;  // first slice of this CTA
     int WS = 0;  // slices: at most one per block, so that none is empty (a unit's slices are then
                  // exactly those from the slice of its first block to that of its last)
     {
         long long base = 0;
         for (int c0 = 0; c0 < B; c0 += CHUNK) {
             const int n = min(CHUNK, B - c0);
-            for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
+            for (int i = threadIdx.x; i < n; i += C::THREADS) {
                 const int c = clamp_context(__ldg(prm.context_lens + c0 + i), cap, blockIdx.x == 0);
                 cum[i] = static_cast<long long>((c + kBlockSize - 1) / kBlockSize) * Hk;
             }
@@ -311,30 +321,35 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             }
             __syncthreads();
             if (B <= CHUNK) N = cum[n - 1];  // one chunk: the total comes with the scan
-            WS = static_cast<int>(min(static_cast<long long>(gridDim.x) * kDecodeWarps, N));
-            for (int i = threadIdx.x; i < n; i += kDecodeThreads) {
+            WS = static_cast<int>(min(static_cast<long long>(gridDim.x) * C::WARPS, N));
+            // a sequence of length 0 has no blocks: CTA b % gridDim.x writes its zero rows
+            for (int i = threadIdx.x; i < n; i += C::THREADS) {
                 const long long hi = cum[i], lo = i ? cum[i - 1] : base;
-                if (lo >= hi) {
-                    // a sequence of length 0 has no blocks: CTA b % gridDim.x writes its zero rows
-                    const int b = c0 + i;
-                    if (b % static_cast<int>(gridDim.x) == static_cast<int>(blockIdx.x)) {
-                        Tq *o = static_cast<Tq *>(prm.out) + static_cast<size_t>(b) * prm.num_heads * D;
-                        for (int e = 0; e < prm.num_heads * D; ++e) store_out(o + e, 0.f);
-                    }
-                    continue;
+                const int b = c0 + i;
+                if (lo >= hi && b % static_cast<int>(gridDim.x) == static_cast<int>(blockIdx.x)) {
+                    Tq *o = static_cast<Tq *>(prm.out) + static_cast<size_t>(b) * prm.num_heads * D;
+                    for (int e = 0; e < prm.num_heads * D; ++e) store_out(o + e, 0.f);
                 }
-#pragma unroll
-                for (int w = 0; w < kDecodeWarps; ++w) {
-                    const long long f = N * (cta0 + w) / max(WS, 1);  // first block of slice cta0 + w
-                    if (cta0 + w < WS && lo <= f && f < hi) {         // ... lies in sequence c0 + i
-                        const int nblk = static_cast<int>((hi - lo) / Hk);
-                        const long long r = f - lo;
-                        starts[5 * w + 0] = c0 + i;
-                        starts[5 * w + 1] = static_cast<int>(r / nblk);
-                        starts[5 * w + 2] = static_cast<int>(r % nblk);
-                        starts[5 * w + 3] = clamp_context(__ldg(prm.context_lens + c0 + i), cap, false);
-                        starts[5 * w + 4] = nblk;
+            }
+            // thread w: the first block of slice cta0 + w, if it lies in this chunk
+            const int w = threadIdx.x;
+            if (w < C::WARPS && cta0 + w < WS) {
+                const long long f = N * (cta0 + w) / WS;
+                if (f >= base && f < cum[n - 1]) {
+                    int lo_i = 0, hi_i = n - 1;  // the first sequence whose inclusive sum exceeds f
+                    while (lo_i < hi_i) {
+                        const int mid = (lo_i + hi_i) / 2;
+                        if (cum[mid] > f) hi_i = mid;
+                        else lo_i = mid + 1;
                     }
+                    const long long lo = lo_i ? cum[lo_i - 1] : base;
+                    const int nblk = static_cast<int>((cum[lo_i] - lo) / Hk);
+                    const long long r = f - lo;
+                    starts[5 * w + 0] = c0 + lo_i;
+                    starts[5 * w + 1] = static_cast<int>(r / nblk);
+                    starts[5 * w + 2] = static_cast<int>(r % nblk);
+                    starts[5 * w + 3] = clamp_context(__ldg(prm.context_lens + c0 + lo_i), cap, false);
+                    starts[5 * w + 4] = nblk;
                 }
             }
             base = cum[n - 1];
@@ -350,6 +365,8 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
 
     unsigned char *ring = smem + warp * C::WARP_RING;
     const uint32_t ring_s = smem_addr(ring);
+    const unsigned char *qslots = smem + C::OFF_Q + warp * C::WARP_Q;
+    const uint32_t q_s = smem_addr(qslots);
     const uint32_t bars = smem_addr(smem + C::OFF_BAR) + warp * C::NSTAGE * 8;
     float *pbuf = reinterpret_cast<float *>(smem + C::OFF_P + warp * C::PBUF);  // [16][G] of (p, p)
     const uint32_t pbuf_s = smem_addr(pbuf);
@@ -367,15 +384,9 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     // (lane i holds block tbase + i)
     int tb_u = -1, tbase = 0, tw = 0;
     uint32_t bad_mask = 0;
-    auto issue = [&](int k, const Cursor &ic) {
+    auto issue = [&](int k, const Cursor &ic, bool new_seg) {
         const int u = ic.b * Hk + ic.hk;
         if (u != tb_u || ic.blk >= tbase + 32) {
-            if (u != tb_u) {  // a new unit: bring its queries towards the SM while its blocks load
-                const char *qrow = static_cast<const char *>(prm.q) +
-                                   (static_cast<size_t>(ic.b) * prm.num_heads + ic.hk * G) * D * sizeof(Tq);
-                if (lane * 128 < G * D * static_cast<int>(sizeof(Tq)))
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + lane * 128));
-            }
             tb_u = u;
             tbase = ic.blk;
             const int e = tbase + lane;
@@ -394,7 +405,12 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         }
         const uint32_t bar = bars + 8 * s;
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+            // the first block of a segment brings the unit's queries along
+            mbar_arrive_expect_tx(bar, C::STAGE_BYTES + (new_seg ? C::QBYTES : 0));
+            if (new_seg)
+                bulk_g2s(q_s + s * C::QBYTES,
+                         static_cast<const Tq *>(prm.q) + (static_cast<size_t>(ic.b) * prm.num_heads + ic.hk * G) * D,
+                         C::QBYTES, bar);
             const uint32_t dst = ring_s + s * C::STAGE_BYTES;
             tma_load_3d(dst, &tm_k, 0, ic.hk, pb * kBlockSize, bar);
             tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar);
@@ -403,18 +419,19 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     {
         Cursor ic = cc;
         for (int i = 0; i < min(C::NSTAGE, nb_w); ++i) {
-            if (i) cursor_advance(ic, 1, prm);
-            issue(i, ic);
+            const bool new_seg = i == 0 || cursor_advance(ic, 1, prm) > 0;
+            issue(i, ic, new_seg);
         }
     }
 
     // Queries of a unit in this lane's head order, pre-scaled by
-    // scale * log2(e), as packed pairs of the lane's columns.
+    // scale * log2(e), as packed pairs of the lane's columns, from the query
+    // slot of stage s.
     f32x2 q2[G][P2];
-    auto load_q = [&](int b, int hk) {
+    auto load_q = [&](int s) {
         constexpr int QV = C::VE * static_cast<int>(sizeof(Tq)) / 16;  // 16-byte q loads per chunk
         constexpr int QP = Widen<Tq>::N / 2;                            // pairs per q load
-        const Tq *qb = static_cast<const Tq *>(prm.q) + (static_cast<size_t>(b) * prm.num_heads + hk * G) * D;
+        const Tq *qb = reinterpret_cast<const Tq *>(qslots + s * C::QBYTES);
         const f32x2 sc = pack2(prm.scale_log2, prm.scale_log2);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -423,7 +440,7 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
             for (int ch = 0; ch < C::CH; ++ch) {
 #pragma unroll
                 for (int u = 0; u < QV; ++u) {
-                    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qh + (ch * C::L + j) * C::VE) + u);
+                    const uint4 raw = *(reinterpret_cast<const uint4 *>(qh + (ch * C::L + j) * C::VE) + u);
                     Widen<Tq>::apply2(raw, &q2[g][ch * VP + u * QP]);
                 }
 #pragma unroll
@@ -531,13 +548,13 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
     bool need_q = true;
     int k = 0;
     for (; k < nb_w; ++k) {
-        if (need_q) {
-            load_q(cc.b, cc.hk);
-            need_q = false;
-        }
         const int s = k % C::NSTAGE;
         const bool landed = mbar_wait(bars + 8 * s, (k / C::NSTAGE) & 1);
         if (!__all_sync(0xffffffffu, landed)) break;
+        if (need_q) {  // the segment's first block: its queries came with it
+            load_q(s);
+            need_q = false;
+        }
         const int last_valid = cc.c - (cc.nblk - 1) * kBlockSize;
         const int n_valid = ((bad_mask >> s) & 1u) ? 0 : (cc.blk == cc.nblk - 1 ? last_valid : kBlockSize);
         unsigned char *kb = ring + s * C::STAGE_BYTES;
@@ -679,8 +696,8 @@ __global__ void __launch_bounds__(kDecodeThreads, DecodeCfg<Tc, D, G>::MIN_BLOCK
         const int passed = k + 1 < nb_w ? cursor_advance(nx, 1, prm) : 0;
         if (k + C::NSTAGE < nb_w) {
             Cursor ic = nx;
-            cursor_advance(ic, C::NSTAGE - 1, prm);
-            issue(k + C::NSTAGE, ic);
+            const bool new_seg = cursor_advance(ic, C::NSTAGE - 1, prm) > 0;  // block k + 2 starts a unit
+            issue(k + C::NSTAGE, ic, new_seg);
         }
         // ---- the last block, or the next one in another unit: the segment closes
         if (passed > 0 || k + 1 == nb_w) {

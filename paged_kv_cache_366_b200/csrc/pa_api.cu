@@ -86,7 +86,7 @@ int resident_of() {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, pa::kDecodeThreads, C::SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, C::THREADS, C::SMEM) != cudaSuccess ||
         n < 1) {
         cudaGetLastError();
         return C::RESIDENT;
@@ -95,29 +95,40 @@ int resident_of() {
     return n;
 }
 
+// CTAs per SM and warps per CTA of the decode kernel for one shape.
+struct DecodeFit {
+    int resident;
+    int warps;
+};
+
+template <typename Tq, typename Tc, int D, int G>
+DecodeFit fit_of() {
+    return DecodeFit{resident_of<Tq, Tc, D, G>(), pa::DecodeCfg<Tc, D, G>::WARPS};
+}
+
 template <typename Tq, typename Tc, int D>
-int resident_g(int g) {
+DecodeFit fit_g(int g) {
     switch (g) {
-        case 1: return resident_of<Tq, Tc, D, 1>();
-        case 2: return resident_of<Tq, Tc, D, 2>();
-        case 4: return resident_of<Tq, Tc, D, 4>();
-        default: return resident_of<Tq, Tc, D, 8>();
+        case 1: return fit_of<Tq, Tc, D, 1>();
+        case 2: return fit_of<Tq, Tc, D, 2>();
+        case 4: return fit_of<Tq, Tc, D, 4>();
+        default: return fit_of<Tq, Tc, D, 8>();
     }
 }
 
-int decode_resident(const pa_shape *s) {
+DecodeFit decode_fit(const pa_shape *s) {
     const int g = s->num_heads / s->num_kv_heads;
     if (s->kv_fp8)
-        return s->head_dim == 128 ? resident_g<__nv_bfloat16, pa::fp8e4m3, 128>(g)
-                                  : resident_g<__nv_bfloat16, pa::fp8e4m3, 64>(g);
+        return s->head_dim == 128 ? fit_g<__nv_bfloat16, pa::fp8e4m3, 128>(g)
+                                  : fit_g<__nv_bfloat16, pa::fp8e4m3, 64>(g);
     if (s->dtype == PA_DTYPE_BF16)
-        return s->head_dim == 128 ? resident_g<__nv_bfloat16, __nv_bfloat16, 128>(g)
-                                  : resident_g<__nv_bfloat16, __nv_bfloat16, 64>(g);
-    return s->head_dim == 128 ? resident_g<float, float, 128>(g) : resident_g<float, float, 64>(g);
+        return s->head_dim == 128 ? fit_g<__nv_bfloat16, __nv_bfloat16, 128>(g)
+                                  : fit_g<__nv_bfloat16, __nv_bfloat16, 64>(g);
+    return s->head_dim == 128 ? fit_g<float, float, 128>(g) : fit_g<float, float, 64>(g);
 }
 
 struct DecodeGeometry {
-    int ctas;          // grid of the persistent decode kernel (kDecodeWarps slices each)
+    int ctas;          // grid of the persistent decode kernel (one slice per warp)
     int64_t slots;     // partial (m, l, O) slots: slice index + unit index
     int64_t ws_bytes;  // workspace bytes
 };
@@ -125,7 +136,7 @@ struct DecodeGeometry {
 int64_t round16(int64_t n) { return (n + 15) / 16 * 16; }
 
 // The decode kernel cuts the flat (sequence, KV head, block) list into
-// 4 * ctas equal slices, one per warp. Automatic: the CTAs all SMs hold at once
+// warps * ctas equal slices, one per warp. Automatic: the CTAs all SMs hold at once
 // (each warp streams one slice; balance comes from equal slices, not from many
 // waves), but no more than one warp per 4 blocks of the largest possible list.
 // With partition_tokens given: slices of about that many tokens of a context
@@ -138,22 +149,22 @@ int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested
     if (requested < 0 || (requested > 0 && (requested % 64 != 0))) return PA_ERR_INVALID_ARGUMENT;
     const int64_t units = static_cast<int64_t>(num_seqs) * s->num_kv_heads;
     const int64_t n_max = units * ((max_context_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+    const DecodeFit fit = decode_fit(s);
     int64_t slices;
     if (requested > 0) {
         slices = (n_max * PA_BLOCK_SIZE + requested - 1) / requested;
     } else {
         const int64_t sms = sm_count() > 0 ? sm_count() : 148;
-        slices = std::min<int64_t>(sms * decode_resident(s) * pa::kDecodeWarps, (n_max + 3) / 4);
+        slices = std::min<int64_t>(sms * fit.resident * fit.warps, (n_max + 3) / 4);
     }
-    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>((slices + pa::kDecodeWarps - 1) / pa::kDecodeWarps,
-                                                                  65535));
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>((slices + fit.warps - 1) / fit.warps, 65535));
     g->ctas = static_cast<int>(ctas);
     if (units == 0) {
         g->slots = 0;
         g->ws_bytes = 0;
     } else {
         const int gq = s->num_heads / s->num_kv_heads;
-        g->slots = ctas * pa::kDecodeWarps + units - 1;
+        g->slots = ctas * fit.warps + units - 1;
         g->ws_bytes = g->slots * gq * s->head_dim * 4 + round16(g->slots * gq * 4) * 2 + round16(units * 8);
     }
     return PA_OK;
@@ -181,7 +192,7 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaSt
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(geo.ctas);
-    cfg.blockDim = dim3(pa::kDecodeThreads);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM;
     cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
     if (e != cudaSuccess) return cuda_fail(e);

@@ -51,11 +51,11 @@ def r16(n):
     return (n + 15) // 16 * 16
 
 
-def ws_bytes(B, ctas, H=32, Hk=8, D=128):
-    """Workspace of a decode over `ctas` CTAs (4 slices each): partial O, m and l per slot (slice + unit),
-    then an int32 (first slice, slices) record per unit."""
+def ws_bytes(B, ctas, H=32, Hk=8, D=128, warps=12):
+    """Workspace of a decode over `ctas` CTAs (one slice per warp, 12 warps for bf16 32/8 heads of 128):
+    partial O, m and l per slot (slice + unit), then an int32 (first slice, slices) record per unit."""
     units = B * Hk
-    slots = 4 * ctas + units - 1
+    slots = warps * ctas + units - 1
     g = H // Hk
     return slots * g * D * 4 + 2 * r16(slots * g * 4) + r16(units * 8)
 
@@ -66,21 +66,22 @@ def test_workspace_sizes():
     assert pa.pa_decode_workspace_bytes(0, 2048, 0, s) == 0
     # one CTA (the list has 8 blocks at most)
     assert pa.pa_decode_workspace_bytes(1, 16, 0, s) == ws_bytes(1, 1)
-    # forced: slices of about 512 tokens of a 2048-token context: 64 * 8 * 128 * 16 / 512 = 2048 slices
-    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == ws_bytes(64, 512)
+    # forced: slices of about 512 tokens of a 2048-token context: 64 * 8 * 128 * 16 / 512 = 2048
+    # slices, 171 CTAs of 12
+    assert pa.pa_decode_workspace_bytes(64, 2048, 512, s) == ws_bytes(64, 171)
     with pytest.raises(pa.PaError):
         pa.pa_decode_workspace_bytes(4, 100, 100, s)  # not a multiple of 64
 
 
 def test_automatic_slices():
-    # no GPU here, so the policy assumes 148 SMs holding 3 decode CTAs each: 444 CTAs, 1776 slices
+    # no GPU here, so the policy assumes 148 SMs holding one decode CTA of 12 warps each: 1776 slices
     from paged_kv_cache_366_b200 import pa
     s = shape()
-    assert pa.pa_decode_workspace_bytes(64, 2048, 0, s) == ws_bytes(64, 444)
-    assert pa.pa_decode_workspace_bytes(8, 32768, 0, s) == ws_bytes(8, 444)
-    assert pa.pa_decode_workspace_bytes(256, 2016, 0, s) == ws_bytes(256, 444)
-    # one sequence of 4096 tokens: 8 * 256 blocks at most, one slice per 4 blocks: 512 slices
-    assert pa.pa_decode_workspace_bytes(1, 4096, 0, s) == ws_bytes(1, 128)
+    assert pa.pa_decode_workspace_bytes(64, 2048, 0, s) == ws_bytes(64, 148)
+    assert pa.pa_decode_workspace_bytes(8, 32768, 0, s) == ws_bytes(8, 148)
+    assert pa.pa_decode_workspace_bytes(256, 2016, 0, s) == ws_bytes(256, 148)
+    # one sequence of 4096 tokens: 8 * 256 blocks at most, one slice per 4 blocks: 512 slices, 43 CTAs
+    assert pa.pa_decode_workspace_bytes(1, 4096, 0, s) == ws_bytes(1, 43)
 
 
 @pytest.mark.parametrize("kw,code", [

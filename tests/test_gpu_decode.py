@@ -83,6 +83,55 @@ def test_long_context_full(pa):
     check_case(pa, W.long_context())
 
 
+# A long ragged list: units of 1 to 1250 blocks, cut by the automatic slicing over every CTA, so
+# that most units are spread over many warps and several CTAs.
+LONG_RAGGED_CTX = [1, 2, 17, 20000, 9000, 3000, 15, 16384, 100, 4097]
+
+
+@pytest.mark.parametrize("dtype,H,Hk,D", [
+    ("bf16", 32, 8, 128), ("bf16", 64, 8, 128), ("bf16", 8, 8, 64), ("f32", 32, 8, 128),
+])
+def test_long_ragged_list(pa, dtype, H, Hk, D):
+    # twice on one workspace of random bytes: the second call starts on the first one's leftovers
+    case = W.make_case("long_ragged", 40 + H + D, context_lens=LONG_RAGGED_CTX, q_lens=[1] * len(LONG_RAGGED_CTX),
+                       num_heads=H, num_kv_heads=Hk, head_dim=D, dtype=dtype)
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    kc_ref, vc_ref = oracle_written(case)
+    ref = oracle.decode(case.q, kc_ref, vc_ref, case.block_tables, case.context_lens, case.scale)
+    mx = int(case.context_lens.max())
+    shape = pa.shape_of(d.k_cache, H)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    ws = torch.randint(0, 256, (pa.pa_decode_workspace_bytes(case.num_seqs, mx, 0, shape),), dtype=torch.uint8,
+                       device="cuda", generator=g)
+    for _ in range(2):
+        out = torch.full_like(d.q, float("nan"))
+        pa.pa_decode(out, d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, 0, ws)
+        assert pa.pa_get_status() == 0
+        err = max_err(to_host(out), ref)
+        assert err <= TOL[dtype], err
+
+
+@pytest.mark.parametrize("partition_tokens", [128, 192, 320, 512, 1024])
+def test_partition_sizes_on_filled_workspace(pa, partition_tokens):
+    # slices of 2 to 17 blocks over units of 1 to 65 blocks: units cut at every kind of place,
+    # on a workspace of 0xff bytes (NaN if any partial or record were read before it is written)
+    ctx = [1, 15, 16, 17, 63, 64, 65, 200, 513, 1000, 1031]
+    case = W.make_case("ragged", 7 + 32 + 128, context_lens=ctx, q_lens=[1] * len(ctx), num_heads=32, num_kv_heads=8,
+                       head_dim=128, dtype="bf16", table_slack=2)
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    kc_ref, vc_ref = oracle_written(case)
+    ref = oracle.decode(case.q, kc_ref, vc_ref, case.block_tables, case.context_lens, case.scale)
+    mx = int(case.context_lens.max())
+    n = pa.pa_decode_workspace_bytes(case.num_seqs, mx, partition_tokens, pa.shape_of(d.k_cache, 32))
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(d.q, float("nan"))
+    pa.pa_decode(out, d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, partition_tokens, ws)
+    assert pa.pa_get_status() == 0
+    assert max_err(to_host(out), ref) <= TOL["bf16"]
+
+
 def test_prefix_sharing_shared_equals_copied(pa):
     a = W.prefix_sharing(copy_shared=False)
     out_a, err_a = check_case(pa, a)
