@@ -452,9 +452,17 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
     def do_write():
         pa.pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, k_scale=ks, v_scale=vs)
 
-    def do_decode():  # one kernel: equal slices of the block list, cut units merged inside
+    def do_decode():  # the partition pass, then the merge of cut units (a programmatic dependent)
         pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws,
                      k_scale=ks, v_scale=vs)
+
+    def do_partials():  # the partition pass alone: decode_kernel, the dominant kernel
+        pa.pa_decode_partials(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0,
+                              ws, k_scale=ks, v_scale=vs)
+
+    def do_merge():  # the merge alone, on the partials the pass before it left in the workspace
+        pa.pa_decode_merge(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0,
+                           ws, k_scale=ks, v_scale=vs)
 
 
     def do_prefill():
@@ -477,7 +485,8 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
             parts.append(("prefill", do_prefill))
         if len(dec):
             parts.append(("decode", do_decode))
-    launches_per_step = len(parts)
+            extra += [("decode_kernel", do_partials), ("merge_kernel", do_merge)]
+    launches_per_step = len(parts) + (1 if len(dec) and not one else 0)  # pa_decode launches two kernels
 
     # one graph for the whole step (the headline), one per part (breakdown, roofline)
     graphs = []
@@ -587,15 +596,20 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
 
 
 def decode_roofline(m, peak, peak_kind, name):
-    """Roofline of the dominant decode kernel: decode_kernel with the fused merge (the pa_decode call)."""
-    t_dec = m["per_part"]["decode"]
+    """Roofline of the dominant decode kernel, decode_kernel (pa_decode_partials, timed alone), with the whole
+    pa_decode call (the kernel and the merge of cut units) beside it."""
+    t_dec = m["per_part"]["decode_kernel"]
+    t_call = m["per_part"]["decode"]
     nb = m["nbytes"]["decode"]
     achieved = nb / t_dec / 1e9
     r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
          "frac_of_nominal": achieved / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
-         "traffic": profiled_traffic(name), "kernel": "decode_kernel (the whole pa_decode call: one launch, "
-                                                      "equal slices per CTA, cut units merged inside)",
+         "traffic": profiled_traffic(name), "kernel": "decode_kernel (pa_decode_partials: the partition pass, "
+                                                      "one CTA of 12 warps per SM, one slice per warp)",
          "algorithmic_bytes_per_launch": nb, "us_per_launch": t_dec * 1e6,
+         "merge_us_per_launch": m["per_part"]["merge_kernel"] * 1e6,
+         "pa_decode_call": {"us": t_call * 1e6, "achieved": nb / t_call / 1e9, "frac": nb / t_call / 1e9 / peak,
+                            "frac_of_nominal": nb / t_call / 1e9 / NOMINAL_HBM_GBS},
          "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else peak_kind}
     return r
 

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 4
+#define PA_ABI_VERSION 5
 #define PA_BLOCK_SIZE 16
 
 typedef enum {
@@ -179,6 +179,25 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
               float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
               const pa_shape *shape, void *stream);
+
+/*
+ * pa_decode_partials, pa_decode_merge: pa_decode's two launches, one call
+ * each, with pa_decode's arguments and checks. pa_decode_partials runs the
+ * partition pass: it writes the output rows of every (sequence, KV head)
+ * whose blocks one warp streamed, and the partials and records of the others
+ * into the workspace. pa_decode_merge, called next on the same stream with
+ * the same arguments and workspace, writes the remaining rows. The pair
+ * gives pa_decode's output bit for bit; other work may run on the stream
+ * between them if it leaves the workspace and out alone.
+ */
+int pa_decode_partials(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                       int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                       void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream);
+int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
+                    int64_t workspace_bytes, const pa_shape *shape, void *stream);
 
 /*
  * pa_prefill_chunk: causal attention for chunks of query tokens placed at a

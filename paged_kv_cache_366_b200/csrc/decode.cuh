@@ -96,7 +96,7 @@ struct DecodeCfg {
     static constexpr int RING_BYTES = WARPS * WARP_RING;
     static constexpr int OFF_Q = RING_BYTES;                // NSTAGE query slots per warp
     static constexpr int OFF_BAR = OFF_Q + WARPS * WARP_Q;  // NSTAGE mbarriers per warp
-    static constexpr int OFF_P = OFF_BAR + WARPS * NSTAGE * 8;
+    static constexpr int OFF_P = OFF_BAR + (WARPS * NSTAGE * 8 + 15) / 16 * 16;
     static constexpr int OFF_MISC = OFF_P + WARPS * PBUF;   // the warps' slice starts
     static constexpr int SMEM = OFF_MISC + WARPS * 5 * 4 + 16;
     // CTAs of this kernel one SM holds, without a device to ask.
@@ -108,7 +108,6 @@ struct DecodeCfg {
     static_assert(OFF_P % 16 == 0 && OFF_MISC % 16 == 0 && QBYTES % 16 == 0, "shared-memory alignment");
     static_assert(STEPS >= 2 && L >= 4, "the first reduce step pairs step slots s and s + STEPS / 2");
     static_assert(SMEM <= kCtaSmem && WARPS >= 1, "one CTA must fit an SM");
-    static_assert(NSTAGE == 2, "the fetch of block k + 2 learns from one step whether it starts a unit");
 };
 
 // Sum, over the lanes that differ in the bits OFF, OFF/2, ..., 1, the N values
@@ -416,12 +415,11 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
             tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar);
         }
     };
-    {
-        Cursor ic = cc;
-        for (int i = 0; i < min(C::NSTAGE, nb_w); ++i) {
-            const bool new_seg = i == 0 || cursor_advance(ic, 1, prm) > 0;
-            issue(i, ic, new_seg);
-        }
+    // the fetch side's cursor: the last block fetched, NSTAGE - 1 ahead of the consumer
+    Cursor icur = cc;
+    for (int i = 0; i < min(C::NSTAGE, nb_w); ++i) {
+        const bool new_seg = i == 0 || cursor_advance(icur, 1, prm) > 0;
+        issue(i, icur, new_seg);
     }
 
     // Queries of a unit in this lane's head order, pre-scaled by
@@ -695,9 +693,8 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
         Cursor nx = cc;  // this warp's next block
         const int passed = k + 1 < nb_w ? cursor_advance(nx, 1, prm) : 0;
         if (k + C::NSTAGE < nb_w) {
-            Cursor ic = nx;
-            const bool new_seg = cursor_advance(ic, C::NSTAGE - 1, prm) > 0;  // block k + 2 starts a unit
-            issue(k + C::NSTAGE, ic, new_seg);
+            const bool new_seg = cursor_advance(icur, 1, prm) > 0;  // block k + NSTAGE starts a unit
+            issue(k + C::NSTAGE, icur, new_seg);
         }
         // ---- the last block, or the next one in another unit: the segment closes
         if (passed > 0 || k + 1 == nb_w) {
@@ -718,31 +715,37 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
 // Merge the partials of every unit cut by slice boundaries:
 //   M = max_s m_s,  L = sum_s 2^(m_s - M) l_s,  out = sum_s 2^(m_s - M) O_s / L
 // over the unit's slices s (slots first + u .. first + slices - 1 + u). Grid
-// (units, G*D/128 column groups); a thread takes four consecutive columns of one
-// head, with every slot's loads of a round in flight together (up to 8 slots a
-// round). A programmatic dependent of decode_kernel: it waits for it before
-// reading the workspace.
-template <typename T, int G, int D>
-__global__ void __launch_bounds__(32) decode_merge_kernel(const DecodeParams prm) {
+// (units, G*D/128 column groups) of MG warps: a lane takes four consecutive
+// columns of one head, warp w the slices w, w + MG, ... with every slot's
+// loads of a round in flight together (up to 8 slots a round); with MG > 1,
+// warp 0 combines the warps' results through shared memory (for units cut
+// into many slices, as in long contexts). A programmatic dependent of
+// decode_kernel: it waits for it before reading the workspace.
+template <typename T, int G, int D, int MG>
+__global__ void __launch_bounds__(32 * MG) decode_merge_kernel(const DecodeParams prm) {
+    __shared__ float4 sh_o[MG][32];
+    __shared__ float sh_m[MG][32], sh_l[MG][32];
     const int u = blockIdx.x;
     const int b = u / prm.num_kv_heads, hk = u % prm.num_kv_heads;
-    const int idx = 4 * (blockIdx.y * 32 + threadIdx.x);
-    if (idx >= G * D) return;
+    const int lane = threadIdx.x % 32, grp = threadIdx.x / 32;
+    const int idx = 4 * (blockIdx.y * 32 + lane);
+    const bool col = idx < G * D;  // the same for every warp: lanes past G * D only take part in the barrier
     if (clamp_context(__ldg(prm.context_lens + b), decode_cap(prm), false) == 0) return;  // zero rows, written
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int first = __ldcg(prm.ws_unit + 2 * u), nseg = __ldcg(prm.ws_unit + 2 * u + 1);
     if (nseg <= 1) return;  // a whole unit: written by the decode kernel
-    const int g = idx / D, d = idx % D;
+    const int g = col ? idx / D : 0, d = col ? idx % D : 0;
     const int s0 = first + u;
     float M = -CUDART_INF_F, Lsum = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = 0; p0 < nseg; p0 += 8) {
+    for (int p0 = grp; p0 < nseg; p0 += 8 * MG) {
         float mp[8], lp[8];
         float4 op[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const bool in = p0 + i < nseg;
-            const size_t s = static_cast<size_t>(s0 + p0 + i);
+            const int p = p0 + i * MG;
+            const bool in = col && p < nseg;
+            const size_t s = static_cast<size_t>(s0 + p);
             mp[i] = in ? __ldcg(prm.ws_m + s * G + g) : -CUDART_INF_F;
             lp[i] = in ? __ldcg(prm.ws_l + s * G + g) : 0.f;
             op[i] = in ? __ldcg(reinterpret_cast<const float4 *>(prm.ws_o + (s * G + g) * D + d))
@@ -770,12 +773,39 @@ __global__ void __launch_bounds__(32) decode_merge_kernel(const DecodeParams prm
         }
         M = mc;
     }
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    O.x *= inv;
-    O.y *= inv;
-    O.z *= inv;
-    O.w *= inv;
-    store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, O);
+    float Lt = Lsum;
+    float4 Ot = O;
+    if constexpr (MG > 1) {
+        sh_o[grp][lane] = O;
+        sh_m[grp][lane] = M;
+        sh_l[grp][lane] = Lsum;
+        __syncthreads();
+        if (grp != 0) return;
+        float Mt = sh_m[0][lane];
+#pragma unroll
+        for (int w = 1; w < MG; ++w) Mt = fmaxf(Mt, sh_m[w][lane]);
+        Lt = 0.f;
+        Ot = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < MG; ++w) {
+            const float mw = sh_m[w][lane];
+            if (mw == -CUDART_INF_F) continue;  // a warp with no slices, or only skipped ones
+            const float wt = exp2f(mw - Mt);
+            const float4 ow = sh_o[w][lane];
+            Ot.x += wt * ow.x;
+            Ot.y += wt * ow.y;
+            Ot.z += wt * ow.z;
+            Ot.w += wt * ow.w;
+            Lt += wt * sh_l[w][lane];
+        }
+    }
+    if (!col) return;
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    Ot.x *= inv;
+    Ot.y *= inv;
+    Ot.z *= inv;
+    Ot.w *= inv;
+    store_out4(static_cast<T *>(prm.out) + (static_cast<size_t>(b) * prm.num_heads + hk * G + g) * D + d, Ot);
 }
 
 }  // namespace pa

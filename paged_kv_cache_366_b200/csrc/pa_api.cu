@@ -170,17 +170,12 @@ int decode_geometry(int32_t num_seqs, int32_t max_context_len, int32_t requested
     return PA_OK;
 }
 
+// The two launches of a decode: the partition pass and the merge.
+enum DecodeParts { kPartials = 1, kMerge = 2, kBoth = 3 };
+
 template <typename Tq, typename Tc, int D, int G>
-int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaStream_t st) {
+int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, int parts, cudaStream_t st) {
     using C = pa::DecodeCfg<Tc, D, G>;
-    resident_of<Tq, Tc, D, G>();  // sets the kernel's shared-memory attributes on this device
-    CUtensorMap tm_k{}, tm_v{};
-    const uint64_t rows = static_cast<uint64_t>(prm.num_blocks) * pa::kBlockSize;
-    if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
-                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
-                       CU_TENSOR_MAP_SWIZZLE_NONE))
-        return PA_ERR_UNSUPPORTED;
     // Both kernels are programmatic dependent launches: each starts launching
     // while the kernel before it drains, and waits for it (griddepcontrol.wait)
     // before reading what it wrote.
@@ -191,25 +186,44 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaSt
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(geo.ctas);
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
-    if (e != cudaSuccess) return cuda_fail(e);
-    cfg.gridDim = dim3(static_cast<unsigned>(prm.num_seqs) * prm.num_kv_heads, (G * D + 127) / 128);
-    cfg.blockDim = dim3(32);
-    cfg.dynamicSmemBytes = 0;
-    e = cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D>, prm);
-    return e == cudaSuccess ? PA_OK : cuda_fail(e);
+    if (parts & kPartials) {
+        resident_of<Tq, Tc, D, G>();  // sets the kernel's shared-memory attributes on this device
+        CUtensorMap tm_k{}, tm_v{};
+        const uint64_t rows = static_cast<uint64_t>(prm.num_blocks) * pa::kBlockSize;
+        if (!pa::encode_3d(&tm_k, prm.k_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
+                           CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !pa::encode_3d(&tm_v, prm.v_cache, D, prm.num_kv_heads, rows, sizeof(Tc), D, 1, pa::kBlockSize,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
+            return PA_ERR_UNSUPPORTED;
+        cfg.gridDim = dim3(geo.ctas);
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (parts & kMerge) {
+        // Four warps per unit when units average 16 slices or more (long
+        // contexts): their slices are merged four ways at once. One otherwise:
+        // fewer, smaller CTAs launch and finish sooner.
+        const int64_t units = static_cast<int64_t>(prm.num_seqs) * prm.num_kv_heads;
+        const bool wide = static_cast<int64_t>(geo.ctas) * C::WARPS >= 16 * units;
+        cfg.gridDim = dim3(static_cast<unsigned>(units), (G * D + 127) / 128);
+        cfg.blockDim = dim3(wide ? 128 : 32);
+        cfg.dynamicSmemBytes = 0;
+        const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 4>, prm)
+                                   : cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 1>, prm);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return PA_OK;
 }
 
 template <typename Tq, typename Tc, int D>
-int dispatch_g(int g, const pa::DecodeParams &prm, const DecodeGeometry &geo, cudaStream_t st) {
+int dispatch_g(int g, const pa::DecodeParams &prm, const DecodeGeometry &geo, int parts, cudaStream_t st) {
     switch (g) {
-        case 1: return launch_decode<Tq, Tc, D, 1>(prm, geo, st);
-        case 2: return launch_decode<Tq, Tc, D, 2>(prm, geo, st);
-        case 4: return launch_decode<Tq, Tc, D, 4>(prm, geo, st);
-        case 8: return launch_decode<Tq, Tc, D, 8>(prm, geo, st);
+        case 1: return launch_decode<Tq, Tc, D, 1>(prm, geo, parts, st);
+        case 2: return launch_decode<Tq, Tc, D, 2>(prm, geo, parts, st);
+        case 4: return launch_decode<Tq, Tc, D, 4>(prm, geo, parts, st);
+        case 8: return launch_decode<Tq, Tc, D, 8>(prm, geo, parts, st);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -281,11 +295,11 @@ int64_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t max_context_len, int
 
 namespace {
 
-// pa_decode after its argument checks.
+// pa_decode (or one of its two launches) after its argument checks.
 int decode_call(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                 int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs, int32_t max_context_len,
                 float scale, int32_t partition_tokens, void *workspace, int64_t workspace_bytes,
-                const pa_shape *shape, void *stream) {
+                const pa_shape *shape, void *stream, int parts = kBoth) {
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARGUMENT;
@@ -332,15 +346,15 @@ int decode_call(void *out, const void *q, const void *k_cache, const void *v_cac
     }
     const int G = shape->num_heads / shape->num_kv_heads;
     if (shape->kv_fp8) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, g, st)
-                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, g, st);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, pa::fp8e4m3, 128>(G, prm, g, parts, st)
+                                      : dispatch_g<__nv_bfloat16, pa::fp8e4m3, 64>(G, prm, g, parts, st);
     }
     if (shape->dtype == PA_DTYPE_BF16) {
-        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, g, st)
-                                      : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, g, st);
+        return shape->head_dim == 128 ? dispatch_g<__nv_bfloat16, __nv_bfloat16, 128>(G, prm, g, parts, st)
+                                      : dispatch_g<__nv_bfloat16, __nv_bfloat16, 64>(G, prm, g, parts, st);
     }
-    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, g, st)
-                                  : dispatch_g<float, float, 64>(G, prm, g, st);
+    return shape->head_dim == 128 ? dispatch_g<float, float, 128>(G, prm, g, parts, st)
+                                  : dispatch_g<float, float, 64>(G, prm, g, parts, st);
 }
 
 }  // namespace
@@ -353,6 +367,22 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               void *stream) {
     return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                        max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream);
+}
+
+int pa_decode_partials(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+                       int32_t num_seqs, int32_t max_context_len, float scale, int32_t partition_tokens,
+                       void *workspace, int64_t workspace_bytes, const pa_shape *shape, void *stream) {
+    return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream, kPartials);
+}
+
+int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                    int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                    int32_t max_context_len, float scale, int32_t partition_tokens, void *workspace,
+                    int64_t workspace_bytes, const pa_shape *shape, void *stream) {
+    return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       max_context_len, scale, partition_tokens, workspace, workspace_bytes, shape, stream, kMerge);
 }
 
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,

@@ -25,7 +25,7 @@ PA_STATUS_BAD_SLOT = 0x2
 PA_STATUS_BAD_CONTEXT = 0x4
 PA_STATUS_WAIT_TIMEOUT = 0x8
 PA_STATUS_BAD_QUERY = 0x10
-PA_ABI_VERSION = 4
+PA_ABI_VERSION = 5
 
 
 class PaShape(ctypes.Structure):
@@ -43,7 +43,8 @@ class PaShape(ctypes.Structure):
 
 
 EXPORTED = [
-    "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_prefill_chunk",
+    "pa_reshape_and_cache", "pa_decode_workspace_bytes", "pa_decode", "pa_decode_partials", "pa_decode_merge",
+    "pa_prefill_chunk",
     "pa_get_status", "pa_strerror", "pa_last_cuda_error", "pa_abi_version", "pa_decode_noalloc",
     "pa_copy_blocks", "pa_swap_blocks",
 ]
@@ -62,8 +63,9 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.restype = ctypes.c_int
     lib.pa_decode_workspace_bytes.argtypes = [I32, I32, I32, SP]
     lib.pa_decode_workspace_bytes.restype = I64
-    lib.pa_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
-    lib.pa_decode.restype = ctypes.c_int
+    for name in ("pa_decode", "pa_decode_partials", "pa_decode_merge"):
+        getattr(lib, name).argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, P, I64, SP, P]
+        getattr(lib, name).restype = ctypes.c_int
     lib.pa_prefill_chunk.argtypes = [P, P, P, P, P, I32, P, P, I32, I32, I32, F, SP, P]
     lib.pa_prefill_chunk.restype = ctypes.c_int
     lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, F, I32, SP, P]
@@ -207,6 +209,22 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
               k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """Decode attention of one query token per sequence over its paged context."""
     _decode("pa_decode", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale)
+
+
+def pa_decode_partials(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+                       partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+                       k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+    """The first of pa_decode's two launches: the partition pass (arguments as pa_decode)."""
+    _decode("pa_decode_partials", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_tokens, workspace, stream, k_scale, v_scale)
+
+
+def pa_decode_merge(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
+                    partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+                    k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+    """The second of pa_decode's two launches: the merge of cut units (arguments as pa_decode)."""
+    _decode("pa_decode_merge", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
             partition_tokens, workspace, stream, k_scale, v_scale)
 
 

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_messages():
     from paged_kv_cache_366_b200 import pa
-    assert pa.pa_abi_version() == 4
+    assert pa.pa_abi_version() == 5
     assert pa.pa_strerror(0) == "ok"
     assert "workspace" in pa.pa_strerror(-4)
     assert pa.pa_strerror(-99) == "unknown error"

@@ -132,6 +132,25 @@ def test_partition_sizes_on_filled_workspace(pa, partition_tokens):
     assert max_err(to_host(out), ref) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("name,part", [("decode_batch", 0), ("long_context", 0), ("decode_batch", 256)])
+def test_partials_then_merge_equals_decode(pa, name, part):
+    # pa_decode's two launches called one by one give its output bit for bit
+    case = W.CONFIGS[name]()
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    mx = int(case.context_lens.max())
+    n = pa.pa_decode_workspace_bytes(case.num_seqs, mx, part, pa.shape_of(d.k_cache, case.num_heads))
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    args = (d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, part, ws)
+    a = torch.full_like(d.q, float("nan"))
+    pa.pa_decode(a, *args)
+    b = torch.full_like(d.q, float("nan"))
+    pa.pa_decode_partials(b, *args)
+    pa.pa_decode_merge(b, *args)
+    assert pa.pa_get_status() == 0
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_prefix_sharing_shared_equals_copied(pa):
     a = W.prefix_sharing(copy_shared=False)
     out_a, err_a = check_case(pa, a)
