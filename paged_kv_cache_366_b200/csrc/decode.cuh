@@ -268,6 +268,18 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
     // waits for this grid to finish before reading anything.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // While the prologue scans the lengths, bring the block tables towards L2
+    // (each CTA a 1/gridDim share, 128-byte lines), so that a warp's first
+    // table read after the prologue does not wait on HBM. Up to 8 MB of table.
+    {
+        const long long lines = (static_cast<long long>(prm.num_seqs) * prm.max_blocks_per_seq * 4 + 127) / 128;
+        if (lines <= (8LL << 20) / 128) {
+            const char *tb = reinterpret_cast<const char *>(prm.block_tables);
+            for (long long i = blockIdx.x + static_cast<long long>(gridDim.x) * threadIdx.x; i < lines;
+                 i += static_cast<long long>(gridDim.x) * C::THREADS)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(tb + i * 128));
+        }
+    }
 
     // ---- prologue (the whole CTA): the total block count N, the slices, and
     // the unit holding each warp's first block, from prefix sums of Hk * blocks
