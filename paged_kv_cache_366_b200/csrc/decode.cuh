@@ -10,13 +10,14 @@
 //
 // How it runs on B200 (two kernels, the second a programmatic dependent):
 //  * Work is the flat list of (sequence, KV head, block) triples in that
-//    order; a (sequence, KV head) pair is a "unit". The grid is persistent
-//    (the CTAs all SMs hold at once) and each warp takes one of
-//    4 * gridDim.x equal, contiguous slices of the list, so every warp gets
-//    the same number of blocks (to one) whatever the mix of lengths: no tail
-//    of short CTAs, no empty CTAs, one prologue per CTA. A CTA finds its
-//    warps' slices by a prefix sum of the sequences' block counts, read from
-//    context_lens on the device. After that the warps run independently.
+//    order; a (sequence, KV head) pair is a "unit". The grid is persistent:
+//    one CTA of WARPS warps per SM (12 for groups of up to 4 heads), and
+//    each warp takes one of WARPS * gridDim.x equal, contiguous slices of
+//    the list, so every warp gets the same number of blocks (to one)
+//    whatever the mix of lengths: no tail of short CTAs, no empty CTAs, one
+//    prologue per CTA. A CTA finds its warps' slices by a prefix sum of the
+//    sequences' block counts, read from context_lens on the device, and one
+//    binary search per warp. After that the warps run independently.
 //  * A unit's part inside one slice is a "segment". A warp leaving a segment
 //    writes the unit's output itself when the whole unit lies in its slice;
 //    otherwise it writes the segment's partial (m, l, O) to the workspace.
@@ -27,7 +28,8 @@
 //    a block's 16 K rows and 16 V rows of one KV head are two TMA tiled loads
 //    (a [16][D] box of the pool viewed as [NB*16][Hk][D]) into a ring slot,
 //    and an mbarrier counts the bytes. Fetches run NSTAGE blocks ahead,
-//    across segment boundaries.
+//    across segment boundaries. The first block of a segment also brings the
+//    unit's G query rows (a bulk copy into the stage's query slot).
 //  * Lanes own column slices of a row made of CH chunks of CB bytes,
 //    interleaved so shared-memory reads are conflict free. L lanes cover a
 //    row and RS = 32 / L rows are processed per step.
