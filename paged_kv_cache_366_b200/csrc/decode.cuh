@@ -172,6 +172,7 @@ struct DecodeParams {
     float *ws_m;   // [slots][G]
     float *ws_l;   // [slots][G]
     int *ws_unit;  // [B][Hk][2]: (first slice, slices) of each unit with blocks, written every call
+    int warps_total;  // the decode kernel's warps (gridDim.x * WARPS): slices = min(warps_total, blocks)
     long long num_blocks;
     int num_seqs;
     int max_blocks_per_seq;
@@ -735,6 +736,10 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
 // warp 0 combines the warps' results through shared memory (for units cut
 // into many slices, as in long contexts). A programmatic dependent of
 // decode_kernel: it waits for it before reading the workspace.
+// Batches of at most this many sequences let each merge CTA find its unit's
+// slices from the lengths before the wait; larger ones read the records.
+constexpr int kMergeScanSeqs = 256;
+
 template <typename T, int G, int D, int MG>
 __global__ void __launch_bounds__(32 * MG) decode_merge_kernel(const DecodeParams prm) {
     __shared__ float4 sh_o[MG][32];
@@ -744,10 +749,39 @@ __global__ void __launch_bounds__(32 * MG) decode_merge_kernel(const DecodeParam
     const int lane = threadIdx.x % 32, grp = threadIdx.x / 32;
     const int idx = 4 * (blockIdx.y * 32 + lane);
     const bool col = idx < G * D;  // the same for every warp: lanes past G * D only take part in the barrier
-    if (clamp_context(__ldg(prm.context_lens + b), decode_cap(prm), false) == 0) return;  // zero rows, written
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int first = __ldcg(prm.ws_unit + 2 * u), nseg = __ldcg(prm.ws_unit + 2 * u + 1);
-    if (nseg <= 1) return;  // a whole unit: written by the decode kernel
+    const int cap = decode_cap(prm);
+    const int c_b = clamp_context(__ldg(prm.context_lens + b), cap, false);
+    if (c_b == 0) return;  // zero rows, written by the decode kernel
+    int first, nseg;
+    if (prm.num_seqs <= kMergeScanSeqs) {
+        // The unit's slices from the lengths alone (inputs, not written by the
+        // decode kernel), before the wait: the same sums as the decode kernel's
+        // prologue. A unit in one slice needs no merge and leaves at once.
+        long long below = 0, total = 0;
+        for (int i = lane; i < prm.num_seqs; i += 32) {
+            const int c = clamp_context(__ldg(prm.context_lens + i), cap, false);
+            const long long n = static_cast<long long>((c + kBlockSize - 1) / kBlockSize) * prm.num_kv_heads;
+            total += n;
+            below += i < b ? n : 0;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            total += __shfl_xor_sync(0xffffffffu, total, off);
+            below += __shfl_xor_sync(0xffffffffu, below, off);
+        }
+        const int nblk = (c_b + kBlockSize - 1) / kBlockSize;
+        const long long u_lo = below + static_cast<long long>(hk) * nblk;
+        const int ws = static_cast<int>(min(static_cast<long long>(prm.warps_total), total));
+        first = slice_of(u_lo, total, ws);
+        nseg = slice_of(u_lo + nblk - 1, total, ws) - first + 1;
+        if (nseg <= 1) return;  // a whole unit: written by the decode kernel
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        first = __ldcg(prm.ws_unit + 2 * u);
+        nseg = __ldcg(prm.ws_unit + 2 * u + 1);
+        if (nseg <= 1) return;  // a whole unit: written by the decode kernel
+    }
     const int g = col ? idx / D : 0, d = col ? idx % D : 0;
     const int s0 = first + u;
     float M = -CUDART_INF_F, Lsum = 0.f;

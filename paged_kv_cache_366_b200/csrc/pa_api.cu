@@ -186,6 +186,8 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, int pa
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    pa::DecodeParams p = prm;
+    p.warps_total = geo.ctas * C::WARPS;
     if (parts & kPartials) {
         resident_of<Tq, Tc, D, G>();  // sets the kernel's shared-memory attributes on this device
         CUtensorMap tm_k{}, tm_v{};
@@ -198,7 +200,7 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, int pa
         cfg.gridDim = dim3(geo.ctas);
         cfg.blockDim = dim3(C::THREADS);
         cfg.dynamicSmemBytes = C::SMEM;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, prm, tm_k, tm_v);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, pa::decode_kernel<Tq, Tc, D, G>, p, tm_k, tm_v);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     if (parts & kMerge) {
@@ -210,8 +212,8 @@ int launch_decode(const pa::DecodeParams &prm, const DecodeGeometry &geo, int pa
         cfg.gridDim = dim3(static_cast<unsigned>(units), (G * D + 127) / 128);
         cfg.blockDim = dim3(wide ? 128 : 32);
         cfg.dynamicSmemBytes = 0;
-        const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 4>, prm)
-                                   : cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 1>, prm);
+        const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 4>, p)
+                                   : cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel<Tq, G, D, 1>, p);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return PA_OK;
