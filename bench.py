@@ -18,8 +18,9 @@ algorithmic bytes over its event time) against the measured HBM copy
 bandwidth, and against the nominal 8000 GB/s. `e2e` times the public
 DecodeStep API from pinned host buffers, with the copies inside.
 `cpu_baseline` is the fp64 oracle on the host cores. On the decode batch the
-line also carries, under `also`, the long-context decode and the prefill
-chunk, each with its own roofline and clocks.
+line also carries, under `also`, the long-context decode, the prefill chunk,
+the FP8 pool, prefix sharing and a batch of verify chunks, each with its own
+roofline and clocks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
@@ -357,6 +358,10 @@ def run_reference(args):
 # sequence (decode tokens as chunks of 1, verify chunks, prefill chunks).
 ONE_LAUNCH = ("varlen_step", "spec_verify")
 NOMINAL_HBM_GBS = 8000.0  # the nominal HBM peak the targets are quoted against
+# Companions of the decode-batch line: the other target config (long context), the tensor-core
+# chunk, the FP8 pool, prefix sharing and a one-launch batch of verify chunks, each timed in the
+# same run with its own roofline and clocks.
+ALSO = ("long_context", "prefill_chunk", "decode_batch_fp8", "prefix_sharing", "spec_verify")
 
 
 def make_workload(name):
@@ -627,6 +632,46 @@ def prefill_roofline(m, name):
             "peak_kind": tkind + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}
 
 
+def one_launch_roofline(m, peak, peak_kind):
+    """One launch does the decode tokens (HBM-bound) and the chunks (tensor-bound when long). Its floor
+    is the chunks' FLOPs at the bf16 peak plus the decode tokens' bytes at the copy bandwidth; a launch
+    of verify chunks alone is HBM-bound (a few rows per KV head)."""
+    case, dec, pre, nbytes = m["case"], m["dec"], m["pre"], m["nbytes"]
+    t_one = m["per_part"]["attention"]
+    tpeak, tkind = load_peak("bf16_tflops")
+    f = prefill_flops(case, pre)
+    attn_bytes = nbytes["decode"] + nbytes["prefill"]
+    long_chunks = [b for b in pre if int(case.q_lens[b]) > 64]
+    f_long = prefill_flops(case, long_chunks)
+    short_bytes = attn_bytes - (step_bytes(case, dec, np.asarray(long_chunks, np.int64))["prefill"]
+                                if long_chunks else 0)
+    t_floor = f_long / (tpeak * 1e12) + short_bytes / (peak * 1e9)
+    roof = {"bound": "hbm" if not long_chunks else "hbm+tensor",
+            "achieved": attn_bytes / t_one / 1e9 if not long_chunks else t_floor / t_one,
+            "peak": peak if not long_chunks else 1.0,
+            "unit": "GB/s" if not long_chunks else "fraction of the summed floor",
+            "frac": t_floor / t_one, "traffic": None,
+            "kernel": "prefill_kernel (tcgen05), one launch over every sequence",
+            "algorithmic_bytes_per_launch": attn_bytes, "flops_per_launch": f,
+            "floor_us": t_floor * 1e6, "us_per_launch": t_one * 1e6,
+            "peak_kind": "%s (MEASURED_PEAKS.json hbm_gbs%s)" % (
+                peak_kind, "" if not long_chunks else " and bf16_tflops, " + tkind)}
+    if not long_chunks:
+        roof["frac_of_nominal"] = attn_bytes / t_one / 1e9 / NOMINAL_HBM_GBS
+    return roof
+
+
+def unique_bytes_entry(m, peak):
+    """Prefix sharing: the decode's K/V bytes counting each shared physical row once."""
+    case, dec, nbytes = m["case"], m["dec"], m["nbytes"]
+    ub = unique_kv_bytes(case, dec) + (nbytes["decode"] - nbytes["kv_decode"])
+    t_dec = m["per_part"]["decode"]
+    return {"decode_bytes": ub, "gbs": ub / t_dec / 1e9, "frac": ub / t_dec / 1e9 / peak,
+            "frac_of_nominal": ub / t_dec / 1e9 / NOMINAL_HBM_GBS,
+            "note": "K/V bytes of the distinct physical rows read (the shared prefix once), "
+                    "plus q, out and tables, over the pa_decode time"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -651,22 +696,27 @@ def run_ours(args):
     value = sum_bytes / t_max / 1e9
     ms_per_step = t_max / args.steps * 1e3
 
-    # companions of the headline in the same run: the other target config of the decode kernel
-    # (long context) and the tensor-core prefill chunk, each with its own roofline and clocks
+    # companions of the headline in the same run (ALSO), each with its own roofline and clocks
     also = {}
     if not args.no_also and args.workload == "decode_batch":
         peak, peak_kind = load_peak()
-        for extra in ("long_context", "prefill_chunk"):
+        for extra in ALSO:
             torch.cuda.empty_cache()
             steps_x = max(5, min(args.steps, 50))
             mx = measure_gpu(extra, steps_x, args.warmup, flush, sampler, want_e2e=False)
             b_x, t_x = aggregate(float(mx["nbytes"]["total"]) * steps_x, mx["total"])
             ent = {"steps": steps_x, "ms_per_step": t_x / steps_x * 1e3, "value": b_x / t_x / 1e9, "unit": UNIT,
+                   "pct_of_hbm_peak": b_x / t_x / 1e9 / peak,
+                   "pct_of_nominal_peak": b_x / t_x / 1e9 / NOMINAL_HBM_GBS,
                    "clocks": mx["clocks"], "config": describe(mx["case"], mx["dec"], mx["pre"])}
-            if len(mx["dec"]):
+            if mx["one"]:
+                ent["roofline"] = one_launch_roofline(mx, peak, peak_kind)
+            elif len(mx["dec"]):
                 ent["roofline"] = decode_roofline(mx, peak, peak_kind, extra)
-            if len(mx["pre"]):
+            elif len(mx["pre"]):
                 ent["roofline"] = prefill_roofline(mx, extra)
+            if extra.startswith("prefix_sharing"):
+                ent["unique_bytes"] = unique_bytes_entry(mx, peak)
             also[extra] = ent
             del mx
 
@@ -713,39 +763,9 @@ def run_ours(args):
             "clocks": m["clocks"], "gpu_launches": m["launches_per_step"] * args.steps,
             "wall_s_timed_region": m["wall"][1] - m["wall"][0]}
     if args.workload.startswith("prefix_sharing"):
-        ub = unique_kv_bytes(case, dec) + (nbytes["decode"] - nbytes["kv_decode"])
-        t_dec = per_part["decode"]
-        line["unique_bytes"] = {"decode_bytes": ub, "gbs": ub / t_dec / 1e9, "frac": ub / t_dec / 1e9 / peak,
-                                "frac_of_nominal": ub / t_dec / 1e9 / NOMINAL_HBM_GBS,
-                                "note": "K/V bytes of the distinct physical rows read (the shared prefix once), "
-                                        "plus q, out and tables, over the pa_decode time"}
+        line["unique_bytes"] = unique_bytes_entry(m, peak)
     if m["one"]:
-        # One launch does the decode tokens (HBM-bound) and the chunks (tensor-bound
-        # when long). Its floor is the chunks' FLOPs at the bf16 peak plus the decode
-        # tokens' bytes at the copy bandwidth; a launch of verify chunks alone is
-        # HBM-bound (a few rows per KV head).
-        t_one = per_part["attention"]
-        tpeak, tkind = load_peak("bf16_tflops")
-        f = prefill_flops(case, pre)
-        attn_bytes = nbytes["decode"] + nbytes["prefill"]
-        long_chunks = [b for b in pre if int(case.q_lens[b]) > 64]
-        f_long = prefill_flops(case, long_chunks)
-        short_bytes = attn_bytes - (step_bytes(case, dec, np.asarray(long_chunks, np.int64))["prefill"]
-                                    if long_chunks else 0)
-        t_floor = f_long / (tpeak * 1e12) + short_bytes / (peak * 1e9)
-        roof = {"bound": "hbm" if not long_chunks else "hbm+tensor",
-                "achieved": attn_bytes / t_one / 1e9 if not long_chunks else t_floor / t_one,
-                "peak": peak if not long_chunks else 1.0,
-                "unit": "GB/s" if not long_chunks else "fraction of the summed floor",
-                "frac": t_floor / t_one, "traffic": None,
-                "kernel": "prefill_kernel (tcgen05), one launch over every sequence",
-                "algorithmic_bytes_per_launch": attn_bytes, "flops_per_launch": f,
-                "floor_us": t_floor * 1e6, "us_per_launch": t_one * 1e6,
-                "peak_kind": "measured (MEASURED_PEAKS.json hbm_gbs%s)" % (
-                    "" if not long_chunks else " and bf16_tflops")}
-        if not long_chunks:
-            roof["frac_of_nominal"] = attn_bytes / t_one / 1e9 / NOMINAL_HBM_GBS
-        line["roofline"] = roof
+        line["roofline"] = one_launch_roofline(m, peak, peak_kind)
     if not m["one"] and len(pre):
         pr = prefill_roofline(m, args.workload)
         line["prefill"] = {"flops": pr["flops_per_launch"], "us_per_launch": pr["us_per_launch"],
