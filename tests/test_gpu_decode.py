@@ -112,6 +112,27 @@ def test_long_ragged_list(pa, dtype, H, Hk, D):
         assert err <= TOL[dtype], err
 
 
+@pytest.mark.parametrize("partition_tokens", [0, 64])
+def test_many_sequences_merge_from_records(pa, partition_tokens):
+    # more than 256 sequences: the merge kernel finds each unit's slices in the records the decode
+    # kernel wrote (fewer sequences let it compute them from the lengths); units cut at every size
+    rng = np.random.default_rng(17)
+    ctx = [int(x) for x in rng.integers(1, 700, size=300)]
+    case = W.make_case("many", 18, context_lens=ctx, q_lens=[1] * len(ctx), num_heads=16, num_kv_heads=4,
+                       head_dim=128, dtype="bf16")
+    d = DevCase(case)
+    pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
+    kc_ref, vc_ref = oracle_written(case)
+    ref = oracle.decode(case.q, kc_ref, vc_ref, case.block_tables, case.context_lens, case.scale)
+    mx = int(case.context_lens.max())
+    n = pa.pa_decode_workspace_bytes(case.num_seqs, mx, partition_tokens, pa.shape_of(d.k_cache, 16))
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(d.q, float("nan"))
+    pa.pa_decode(out, d.q, d.k_cache, d.v_cache, d.block_tables, d.context_lens, mx, case.scale, partition_tokens, ws)
+    assert pa.pa_get_status() == 0
+    assert max_err(to_host(out), ref) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("partition_tokens", [128, 192, 320, 512, 1024])
 def test_partition_sizes_on_filled_workspace(pa, partition_tokens):
     # slices of 2 to 17 blocks over units of 1 to 65 blocks: units cut at every kind of place,
