@@ -66,7 +66,7 @@ struct DecodeCfg {
     // per chunk as for bf16 (16 would spill q and O).
     static constexpr int CB = E == 1 ? 8 : 16;
     // One chunk per lane and row: q and O then take 64 registers for 4 heads
-    // (two chunks spill at three CTAs per SM).
+    // (two chunks spill at 12 warps per SM).
     static constexpr int CH = 1;
     static constexpr int L = R / (CB * CH);                // lanes covering one row
     static constexpr int RS = 32 / L;                      // rows per warp step
@@ -75,8 +75,8 @@ struct DecodeCfg {
     static constexpr int EPL = CH * VE;                    // elements per lane per row
     static constexpr int P2 = EPL / 2;                     // packed pairs per lane per row
     static constexpr int STAGE_BYTES = 2 * kBlockSize * R; // K and V of one block
-    // Two stages per warp and three CTAs per SM (12 warps) measured faster on
-    // B200 than three stages at two CTAs per SM.
+    // Two stages per warp at 12 warps per SM measured faster on B200 than
+    // three stages at 8 warps or four at 6 (the same bytes in flight).
     static constexpr int NSTAGE = 2;
     static constexpr int WARP_RING = NSTAGE * STAGE_BYTES;
     static constexpr int NPART = STEPS * G;                 // q.k partials per lane per block
