@@ -89,7 +89,8 @@ LONG_RAGGED_CTX = [1, 2, 17, 20000, 9000, 3000, 15, 16384, 100, 4097]
 
 
 @pytest.mark.parametrize("dtype,H,Hk,D", [
-    ("bf16", 32, 8, 128), ("bf16", 64, 8, 128), ("bf16", 8, 8, 64), ("f32", 32, 8, 128),
+    ("bf16", 32, 8, 128), ("bf16", 64, 8, 128), ("bf16", 8, 8, 64), ("f32", 32, 8, 128), ("bf16", 16, 8, 128),
+    ("f32", 16, 8, 64),
 ])
 def test_long_ragged_list(pa, dtype, H, Hk, D):
     # twice on one workspace of random bytes: the second call starts on the first one's leftovers

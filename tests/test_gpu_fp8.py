@@ -85,6 +85,15 @@ def test_fp8_ragged(pa, H, Hk, D, partition_tokens):
     check_fp8_decode(pa, case, partition_tokens)
 
 
+@pytest.mark.parametrize("H,Hk", [(32, 8), (64, 8)])
+def test_fp8_long_ragged_list(pa, H, Hk):
+    # units of 1 to 1250 blocks spread over every CTA: the merge runs four warps per unit
+    ctx = [1, 2, 17, 20000, 9000, 3000, 15, 16384, 100, 4097]
+    case = W.make_case("fp8long", 80 + H, context_lens=ctx, q_lens=[1] * len(ctx), num_heads=H, num_kv_heads=Hk,
+                       head_dim=128, dtype="bf16")
+    check_fp8_decode(pa, case)
+
+
 def test_fp8_prefill_is_refused(pa):
     kc = torch.zeros((4, 16, 8, 128), dtype=torch.uint8, device="cuda")
     q = torch.zeros((2, 32, 128), dtype=torch.bfloat16, device="cuda")
