@@ -75,26 +75,66 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 x bf16 -> fp32, one thread issues.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// The eight K=16 steps of one tile's MMA, issued by one thread from one asm
+// block. A shared-memory descriptor addresses 16-byte units in its low 14 bits,
+// so the descriptor of base + off is the base's descriptor plus off / 16 (no
+// carry below 256 KB): each step adds a constant instead of rebuilding both
+// descriptors.
+
+// S = Q K^T over head_dim 128: a and b describe the first step of Q and K
+// (K-major, 128-byte swizzle, 64-column halves 16 KB apart; step kk advances
+// (kk / 4) * 16 KB + (kk % 4) * 32 B). The first step overwrites S.
+__device__ __forceinline__ void umma_qk_d128(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred pf, pt;\n\t.reg .b64 a1, b1;\n\t"
+        "setp.ne.b32 pf, %3, %3;\n\t"
+        "setp.eq.b32 pt, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 4;\n\tadd.s64 b1, %2, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 6;\n\tadd.s64 b1, %2, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 1024;\n\tadd.s64 b1, %2, 1024;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 1026;\n\tadd.s64 b1, %2, 1026;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 1028;\n\tadd.s64 b1, %2, 1028;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "add.s64 a1, %1, 1030;\n\tadd.s64 b1, %2, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc)
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]: the A operand (M rows = TMEM lanes, K
-// along columns, two bf16 per 32-bit column) is read from tensor memory.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// O (+)= P V over 128 keys: P, the A operand, is read from tensor memory (16
+// keys = 8 columns per step); b describes V's first 16 keys (MN-major, 2 KB per
+// 16 keys). The first step accumulates iff `accumulate`.
+__device__ __forceinline__ void umma_pv_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                              uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred pa, pt;\n\t.reg .b32 a1;\n\t.reg .b64 b1;\n\t"
+        "setp.ne.b32 pa, %4, 0;\n\t"
+        "setp.eq.b32 pt, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, pa;\n\t"
+        "add.s32 a1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 16;\n\tadd.s64 b1, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 24;\n\tadd.s64 b1, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 32;\n\tadd.s64 b1, %2, 512;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 40;\n\tadd.s64 b1, %2, 640;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 48;\n\tadd.s64 b1, %2, 768;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "add.s32 a1, %1, 56;\n\tadd.s64 b1, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, pt;\n\t"
+        "}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -482,25 +522,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 auto issue_qk = [&](int qi, int j) {  // S_qi = Q K_j^T
                     const uint32_t qb = base_s + kPfOffQ + (split ? 0 : qi) * kPfQTile;
                     const uint32_t kb = base_s + kPfOffK + (j % kPfNSK) * kPfKVTile;
-#pragma unroll
-                    for (int kk = 0; kk < kPfD / 16; ++kk) {
-                        umma_bf16(tmem + qi * kPfN,
-                                  smem_desc_sw128(qb + (kk >> 2) * kPfQHalf + (kk & 3) * 32, 16, 1024),
-                                  smem_desc_sw128(kb + (kk >> 2) * kPfKVHalf + (kk & 3) * 32, 16, 1024), kIdQK,
-                                  kk > 0);
-                    }
+                    static_assert(kPfQHalf == 16384 && kPfKVHalf == 16384 && kPfD == 128, "umma_qk_d128 steps");
+                    umma_qk_d128(tmem + qi * kPfN, smem_desc_sw128(qb, 16, 1024), smem_desc_sw128(kb, 16, 1024),
+                                 kIdQK);
                     umma_commit(b_tile(qi, 0));
                     if (last(qi)) umma_commit(bar(kPfBarKE + j % kPfNSK));
                 };
                 auto issue_pv = [&](int qi, int j, bool acc) {  // O_qi (+)= P_qi V_j, P read from tensor memory
                     const uint32_t pt = tmem + qi * kPfN + kPfColP;
                     const uint32_t vb = base_s + kPfOffV + (j % kPfNSV) * kPfKVTile;
-#pragma unroll
-                    for (int kk = 0; kk < kPfN / 16; ++kk) {  // 16 keys = 8 columns of P
-                        umma_bf16_ts(tmem + kPfColO + qi * kPfD, pt + kk * 8,
-                                     smem_desc_sw128(vb + kk * 2048, kPfKVHalf, 1024), kIdPV,
-                                     (acc || kk > 0) ? 1u : 0u);
-                    }
+                    static_assert(kPfN == 128, "umma_pv_k128 covers 128 keys");
+                    umma_pv_k128(tmem + kPfColO + qi * kPfD, pt, smem_desc_sw128(vb, kPfKVHalf, 1024), kIdPV,
+                                 acc ? 1u : 0u);
                     umma_commit(b_tile(qi, 2));
                     if (last(qi)) umma_commit(bar(kPfBarVE + j % kPfNSV));
                 };
