@@ -121,6 +121,27 @@ def test_null_pointers_are_rejected_before_any_launch():
     assert rc == -2  # prefill is bf16 only
 
 
+def test_empty_inputs_are_no_ops():
+    """Empty batches return success before any check that needs a pointer, and launch nothing (the
+    calls below run on a machine without a GPU)."""
+    from paged_kv_cache_366_b200 import pa
+    s = shape()
+    by = ctypes.byref(s)
+    assert pa.lib.pa_reshape_and_cache(None, None, None, None, None, 0, by, None) == 0
+    for fn in (pa.lib.pa_decode, pa.lib.pa_decode_partials, pa.lib.pa_decode_merge):
+        assert fn(None, None, None, None, None, 4, None, 0, 64, 1.0, 0, None, 0, by, None) == 0
+    assert pa.lib.pa_decode_noalloc(None, None, None, None, None, 4, None, 0, 64, 1.0, 0, by, None) == 0
+    # no sequences, or sequences with no query tokens
+    assert pa.lib.pa_prefill_chunk(None, None, None, None, None, 4, None, None, 0, 8, 8, 1.0, by, None) == 0
+    assert pa.lib.pa_prefill_chunk(None, None, None, None, None, 4, None, None, 2, 0, 0, 1.0, by, None) == 0
+    assert pa.lib.pa_copy_blocks(None, None, None, 0, by, None) == 0
+    assert pa.lib.pa_swap_blocks(None, None, None, 0, 4, 4, 16 * 8 * 128 * 2, None) == 0
+    # negative sizes are errors, not no-ops
+    assert pa.lib.pa_reshape_and_cache(None, None, None, None, None, -1, by, None) == -1
+    assert pa.lib.pa_decode(None, None, None, None, None, 4, None, -1, 64, 1.0, 0, None, 0, by, None) == -1
+    assert pa.lib.pa_copy_blocks(None, None, None, -1, by, None) == -1
+
+
 def test_misaligned_pointer_is_rejected():
     from paged_kv_cache_366_b200 import pa
     s = shape()
