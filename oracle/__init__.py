@@ -66,6 +66,8 @@ def _load():
             lib.pa_oracle_reshape_and_cache_fp8.restype = L
             lib.pa_oracle_decode_fp8.argtypes = [P, P, I, P, P, D, D, P, I, P, I, I, I, I, I, L, D, I]
             lib.pa_oracle_decode_fp8.restype = I
+            lib.pa_oracle_prefill_fp8.argtypes = [P, P, I, P, P, D, D, P, I, P, P, I, I, I, I, I, L, D, P, L, I]
+            lib.pa_oracle_prefill_fp8.restype = I
             lib.pa_oracle_set_mutation.argtypes = [I]
             lib.pa_oracle_set_mutation.restype = None
             lib.pa_oracle_get_mutation.argtypes = []
@@ -270,4 +272,32 @@ def decode_fp8(q, k_cache, v_cache, k_scale: float, v_scale: float, block_tables
                                       bs, NB, float(scale), int(num_threads))
     if rc:
         raise OracleError("decode failed (%d)" % rc)
+    return out
+
+
+def prefill_fp8(q, k_cache, v_cache, k_scale: float, v_scale: float, block_tables, cu_q_lens, context_lens,
+                scale: float, rows=None, num_threads: int = 0):
+    """Causal chunk attention over E4M3 caches (uint8 codes): K, V = code value times k_scale, v_scale.
+    out [T or len(rows), H, D] fp64."""
+    q = _c(q)
+    k_cache = _c(k_cache, np.uint8)
+    v_cache = _c(v_cache, np.uint8)
+    bt = _c(block_tables, np.int32)
+    cu = _c(cu_q_lens, np.int32)
+    cl = _c(context_lens, np.int32)
+    T, H, D = q.shape
+    NB, bs, Hk, D2 = k_cache.shape
+    B = cl.shape[0]
+    assert D == D2 and cu.shape[0] == B + 1 and int(cu[-1]) == T and bt.shape[0] == B
+    if rows is None:
+        n_rows, rows_p = T, None
+    else:
+        rows_arr = _c(rows, np.int32)
+        n_rows, rows_p = rows_arr.shape[0], _ptr(rows_arr)
+    out = np.zeros((n_rows, H, D), np.float64)
+    rc = _load().pa_oracle_prefill_fp8(_ptr(out), _ptr(q), _dtype_code(q), _ptr(k_cache), _ptr(v_cache),
+                                       float(k_scale), float(v_scale), _ptr(bt), bt.shape[1], _ptr(cu), _ptr(cl), B, H,
+                                       Hk, D, bs, NB, float(scale), rows_p, n_rows, int(num_threads))
+    if rc:
+        raise OracleError("prefill failed (%d)" % rc)
     return out

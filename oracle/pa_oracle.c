@@ -291,11 +291,11 @@ int pa_oracle_decode(double *out, const void *q, const void *k_cache, const void
  * out is [T][H][D]. Otherwise out is [n_rows][H][D], holding the listed
  * global rows in order. Returns 0, -1 or -2 as decode does.
  */
-int pa_oracle_prefill(double *out, const void *q, const void *k_cache, const void *v_cache, int dtype,
-                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *cu_q_lens,
-                      const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
-                      int head_dim, int block_size, long num_blocks, double scale,
-                      const int32_t *rows, long n_rows, int num_threads)
+static int prefill_impl(double *out, const void *q, int q_dtype, const void *k_cache, const void *v_cache,
+                        int kv_dtype, double k_scale, double v_scale, const int32_t *block_tables,
+                        int max_blocks_per_seq, const int32_t *cu_q_lens, const int32_t *context_lens,
+                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                        long num_blocks, double scale, const int32_t *rows, long n_rows, int num_threads)
 {
     if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return -2;
@@ -334,12 +334,18 @@ int pa_oracle_prefill(double *out, const void *q, const void *k_cache, const voi
         double *Vc = malloc(sizeof(double) * (size_t)(c > 0 ? c : 1) * head_dim);
         double *s = malloc(sizeof(double) * (size_t)(c > 0 ? c : 1));
         double *qv = malloc(sizeof(double) * (size_t)head_dim);
-        int rc = pa_oracle_gather(Kc, Vc, k_cache, v_cache, dtype, block_tables, max_blocks_per_seq, b,
+        int rc = pa_oracle_gather(Kc, Vc, k_cache, v_cache, kv_dtype, block_tables, max_blocks_per_seq, b,
                                   c, num_kv_heads, hk, head_dim, block_size, num_blocks);
         if (rc) {
 #pragma omp critical
             status = rc;
         } else {
+            if (kv_dtype == ORACLE_FP8_E4M3) {
+                for (long i = 0; i < c * head_dim; ++i) {
+                    Kc[i] *= k_scale;
+                    Vc[i] *= v_scale;
+                }
+            }
             for (long i = 0; i < n_rows; ++i) {
                 long r = rows ? rows[i] : i;
                 if (r < q0 || r >= q1)
@@ -356,7 +362,7 @@ int pa_oracle_prefill(double *out, const void *q, const void *k_cache, const voi
                         continue;
                     long qbase = (r * num_heads + h) * (long)head_dim;
                     for (int d = 0; d < head_dim; ++d)
-                        qv[d] = load_elem(q, qbase + d, dtype);
+                        qv[d] = load_elem(q, qbase + d, q_dtype);
                     attend(out + (i * num_heads + h) * (long)head_dim, qv, Kc, Vc, n_keys, head_dim,
                            scale, s);
                 }
@@ -368,6 +374,33 @@ int pa_oracle_prefill(double *out, const void *q, const void *k_cache, const voi
         free(qv);
     }
     return status;
+}
+
+int pa_oracle_prefill(double *out, const void *q, const void *k_cache, const void *v_cache, int dtype,
+                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *cu_q_lens,
+                      const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, long num_blocks, double scale,
+                      const int32_t *rows, long n_rows, int num_threads)
+{
+    return prefill_impl(out, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0, block_tables, max_blocks_per_seq,
+                        cu_q_lens, context_lens, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                        num_blocks, scale, rows, n_rows, num_threads);
+}
+
+/*
+ * Prefill chunk over FP8 E4M3 caches: K = e4m3(code) * k_scale, V =
+ * e4m3(code) * v_scale, q and out as q_dtype. Otherwise identical to
+ * pa_oracle_prefill.
+ */
+int pa_oracle_prefill_fp8(double *out, const void *q, int q_dtype, const uint8_t *k_cache,
+                          const uint8_t *v_cache, double k_scale, double v_scale, const int32_t *block_tables,
+                          int max_blocks_per_seq, const int32_t *cu_q_lens, const int32_t *context_lens,
+                          int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                          long num_blocks, double scale, const int32_t *rows, long n_rows, int num_threads)
+{
+    return prefill_impl(out, q, q_dtype, k_cache, v_cache, ORACLE_FP8_E4M3, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, cu_q_lens, context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale, rows, n_rows, num_threads);
 }
 
 /*

@@ -79,6 +79,46 @@ def test_fp8_decode_equals_attention_over_dequantized_cache():
     assert np.array_equal(got, ref)
 
 
+def test_fp8_prefill_equals_attention_over_dequantized_cache():
+    # ragged chunks at offsets (one of them a single decode token, one a whole prompt)
+    case = W.make_case("fp8p", 222, context_lens=[40, 37, 100, 300], q_lens=[40, 1, 23, 70], num_heads=8,
+                       num_kv_heads=2, head_dim=64, dtype="bf16")
+    kc_bf, vc_bf = oracle.reshape_and_cache(case.k_new, case.v_new, case.k_cache, case.v_cache, case.slot_mapping)
+    case.k_cache, case.v_cache = kc_bf, vc_bf
+    ks, vs = 0.5, 0.25  # powers of two: dequantized values are exact in fp32
+    kc, vc = _fp8_pool(case, ks, vs)
+    got = oracle.prefill_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.cu_q_lens, case.context_lens,
+                             case.scale)
+    deq = np.vectorize(oracle.e4m3_decode)
+    kf = (deq(kc) * ks).astype(np.float32)
+    vf = (deq(vc) * vs).astype(np.float32)
+    qf = W.bf16_bits_to_f32(case.q)
+    ref = oracle.prefill(qf, kf, vf, case.block_tables, case.cu_q_lens, case.context_lens, case.scale)
+    assert np.isfinite(ref).all() and np.array_equal(got, ref)
+    # the scales are not interchangeable: K's scale sharpens the softmax, V's scales the output
+    swapped = oracle.prefill_fp8(case.q, kc, vc, vs, ks, case.block_tables, case.cu_q_lens, case.context_lens,
+                                 case.scale)
+    assert not np.allclose(swapped, got)
+    # a subset of rows gives the same rows
+    rows = np.array([0, 39, 40, 41, 63, 64, 133], np.int32)
+    sub = oracle.prefill_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.cu_q_lens, case.context_lens,
+                             case.scale, rows=rows)
+    assert np.array_equal(sub, got[rows])
+
+
+def test_fp8_prefill_of_single_tokens_equals_fp8_decode():
+    case = W.make_case("fp8p1", 223, context_lens=[1, 16, 17, 250], q_lens=[1] * 4, num_heads=8, num_kv_heads=2,
+                       head_dim=64, dtype="bf16")
+    kc_bf, vc_bf = oracle.reshape_and_cache(case.k_new, case.v_new, case.k_cache, case.v_cache, case.slot_mapping)
+    case.k_cache, case.v_cache = kc_bf, vc_bf
+    ks, vs = 0.02, 1.0 / 48.0
+    kc, vc = _fp8_pool(case, ks, vs)
+    dec = oracle.decode_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.context_lens, case.scale)
+    pre = oracle.prefill_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.cu_q_lens, case.context_lens,
+                             case.scale)
+    assert np.isfinite(dec).all() and np.array_equal(pre, dec)
+
+
 def test_fp8_write_quantizes_in_fp32_then_rounds():
     k = W.f32_to_bf16_bits(np.array([[[0.3, -0.77, 1.0, 0.0]]], np.float32))
     kc = np.zeros((2, 16, 1, 4), np.uint8)
