@@ -53,7 +53,7 @@ FLUSH_BYTES = 256 << 20
 DECODE_SOURCES = ["decode.cuh", "pa_common.cuh", "tmap.cuh"]
 PREFILL_SOURCES = ["prefill_sm100.cuh", "pa_common.cuh", "tmap.cuh"]
 WORKLOADS = ["decode_batch", "long_context", "prefix_sharing", "mixed_step", "prefill_chunk", "tiny",
-             "copy_blocks", "swap_blocks", "decode_batch_fp8", "varlen_step", "spec_verify"]
+             "copy_blocks", "swap_blocks", "decode_batch_fp8", "prefill_chunk_fp8", "varlen_step", "spec_verify"]
 FP8_K_SCALE, FP8_V_SCALE = 0.02, 1.0 / 48.0
 BLOCK_WORKLOADS = ("copy_blocks", "swap_blocks")
 BLOCK_PAIRS = 2048
@@ -361,12 +361,12 @@ NOMINAL_HBM_GBS = 8000.0  # the nominal HBM peak the targets are quoted against
 # Companions of the decode-batch line: the other target config (long context), the tensor-core
 # chunk, the FP8 pool, prefix sharing and a one-launch batch of verify chunks, each timed in the
 # same run with its own roofline and clocks.
-ALSO = ("long_context", "prefill_chunk", "decode_batch_fp8", "prefix_sharing", "spec_verify")
+ALSO = ("long_context", "prefill_chunk", "decode_batch_fp8", "prefill_chunk_fp8", "prefix_sharing", "spec_verify")
 
 
 def make_workload(name):
-    if name == "decode_batch_fp8":
-        return W.decode_batch()
+    if name.endswith("_fp8"):  # the same sequences over a pool of E4M3 codes
+        name = name[:-len("_fp8")]
     if name == "varlen_step":  # the mixed step's sequences, attended in one launch
         return W.mixed_step()
     if name not in W.CONFIGS:
@@ -417,7 +417,7 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
 
     case = make_workload(name)
     dec, pre = split_seqs(case)
-    fp8 = name == "decode_batch_fp8"
+    fp8 = name.endswith("_fp8")
     ks, vs = (FP8_K_SCALE, FP8_V_SCALE) if fp8 else (0.0, 0.0)
     nbytes = step_bytes(case, dec, pre, 1 if fp8 else None)
 
@@ -473,14 +473,15 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
 
     def do_prefill():
         pa.pa_prefill_chunk(out_pre, q_pre, k_cache, v_cache, tables[p0:p1], cu_pre, lens[p0:p1], max_q,
-                            case.scale)
+                            case.scale, k_scale=ks, v_scale=vs)
 
     one = name in ONE_LAUNCH
     out_all = torch.empty_like(q)
     max_q_all = int(case.q_lens.max())
 
     def do_all():  # every sequence's chunk, decode tokens included, in one launch
-        pa.pa_prefill_chunk(out_all, q, k_cache, v_cache, tables, cu, lens, max_q_all, case.scale)
+        pa.pa_prefill_chunk(out_all, q, k_cache, v_cache, tables, cu, lens, max_q_all, case.scale, k_scale=ks,
+                            v_scale=vs)
 
     parts = [("write", do_write)]
     extra = []
@@ -709,6 +710,9 @@ def run_ours(args):
                    "pct_of_hbm_peak": b_x / t_x / 1e9 / peak,
                    "pct_of_nominal_peak": b_x / t_x / 1e9 / NOMINAL_HBM_GBS,
                    "clocks": mx["clocks"], "config": describe(mx["case"], mx["dec"], mx["pre"])}
+            if mx["fp8"]:
+                ent["config"].update({"workload": extra, "kv_dtype": "fp8_e4m3", "k_scale": mx["ks"],
+                                      "v_scale": mx["vs"]})
             if mx["one"]:
                 ent["roofline"] = one_launch_roofline(mx, peak, peak_kind)
             elif len(mx["dec"]):
@@ -744,7 +748,7 @@ def run_ours(args):
     parts_ms = {k: v * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
     if m["fp8"]:
-        config.update({"workload": "decode_batch_fp8", "kv_dtype": "fp8_e4m3", "k_scale": m["ks"],
+        config.update({"workload": args.workload, "kv_dtype": "fp8_e4m3", "k_scale": m["ks"],
                        "v_scale": m["vs"]})
     config.update({"l2": "flushed before every step and every timed part, outside the events: 256 MiB memset, "
                          "then a 256 MiB read so the memset's write-back is not charged to the step",

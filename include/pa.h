@@ -93,9 +93,9 @@ typedef struct {
      * infinities, largest finite 448). A cached value means code * k_scale
      * (keys) or code * v_scale (values). The write quantizes
      * fp32(x) * fp32(1 / scale) to the nearest code (ties to even, saturating
-     * at +-448). FP8 caches need dtype = PA_DTYPE_BF16; pa_prefill_chunk does
-     * not take them. The pages name FP8 only for weights ("vLLM and
-     * PagedAttention" §5); an FP8 cache halves the bytes decode reads.
+     * at +-448). FP8 caches need dtype = PA_DTYPE_BF16. The pages name FP8
+     * only for weights ("vLLM and PagedAttention" §5); an FP8 cache halves the
+     * bytes decode reads.
      */
     int32_t kv_fp8;
     float k_scale; /* > 0 when kv_fp8; ignored otherwise */
@@ -219,9 +219,15 @@ int pa_decode_merge(void *out, const void *q, const void *k_cache, const void *v
  *   max_q_len    : host-side upper bound of every q_len (checked, >= 0; the
  *                  grid is sized from num_q_tokens and num_seqs)
  *   scale        : softmax scale, > 0 (PA_ERR_INVALID_ARGUMENT otherwise)
- * bf16 only, D = 128 only. Runs on the tcgen05 tensor cores with fp32
- * accumulation in tensor memory. Probabilities enter P.V rounded to bf16;
- * the row sums use them unrounded. Returns PA_ERR_UNSUPPORTED otherwise.
+ * q and out bf16, D = 128 only; the caches bf16, or FP8 E4M3 codes
+ * (kv_fp8 = 1). Runs on the tcgen05 tensor cores with fp32 accumulation in
+ * tensor memory. Probabilities enter P.V rounded to bf16; the row sums use
+ * them unrounded. Over an FP8 pool the MMAs take f16 operands: each K/V tile's
+ * codes are widened exactly to f16 in shared memory, q is rounded to f16 there
+ * (exact for |q| in [2^-14, 65504] and for 0; outside that range q is rounded
+ * or saturates to infinity), P enters P.V rounded to f16, k_scale joins the
+ * softmax scale and v_scale the output. Returns PA_ERR_UNSUPPORTED for other
+ * shapes.
  */
 int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *cu_q_lens,

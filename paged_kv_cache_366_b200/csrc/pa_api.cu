@@ -391,7 +391,6 @@ int pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *
                      int32_t max_blocks_per_seq, const int32_t *cu_q_lens, const int32_t *context_lens,
                      int32_t num_seqs, int32_t max_q_len, int32_t num_q_tokens, float scale, const pa_shape *shape,
                      void *stream) {
-    if (shape && shape->kv_fp8) return PA_ERR_UNSUPPORTED;  // FP8 caches are a decode-only layout
     int rc = check_shape(shape);
     if (rc != PA_OK) return rc;
     if (shape->dtype != PA_DTYPE_BF16 || shape->head_dim != 128) return PA_ERR_UNSUPPORTED;

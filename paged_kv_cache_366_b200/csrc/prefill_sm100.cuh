@@ -43,6 +43,11 @@
 //    replaced (and O rescaled in TMEM) only when a row max grows by more than
 //    2^8, so the first half is exponentiated before the second is read, and
 //    only re-scaled in the rare case that the second half moves m.
+//  * Over an FP8 (E4M3) pool the producers TMA-load each tile's codes into a
+//    staging buffer and widen them exactly to f16 into the stage (one
+//    cvt.rn.f16x2.e4m3x2 per pair), so the MMAs take f16 operands: q is
+//    converted to f16 in shared memory once per CTA and P is written as f16.
+//    k_scale joins the softmax scale and v_scale the output.
 //  * Hand-offs are mbarriers only: full/empty per ring stage (empties committed
 //    by tcgen05.commit), and per Q tile sfull (S ready; it also implies the
 //    previous P V is done, so O may be rescaled), pready and odone. Every wait
@@ -50,6 +55,7 @@
 //    drains its work before tensor memory is freed.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include <atomic>
@@ -214,10 +220,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A K-major,
-// B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16 or
+// both f16, A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int b_mn, bool f16) {
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | (static_cast<uint32_t>(b_mn) << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -232,23 +238,37 @@ constexpr int kPfNQ = 2;                     // Q tiles per CTA, ping-ponged
 constexpr int kPfN = 128;                    // keys per K/V tile
 constexpr int kPfD = 128;                    // head_dim
 constexpr int kPfNSK = 2;                    // K pipeline stages
-constexpr int kPfNSV = 3;                    // V pipeline stages (a V tile is held longest)
 constexpr int kPfQHalf = kPfM * 64 * 2;      // a 64-column half of a Q tile: 16 KB
 constexpr int kPfQTile = 2 * kPfQHalf;       // 32 KB
 constexpr int kPfKVHalf = kPfN * 64 * 2;     // a 64-dim half of a K/V tile: 16 KB
 constexpr int kPfKVTile = 2 * kPfKVHalf;     // 32 KB
 constexpr int kPfOffQ = 0;
 constexpr int kPfOffK = kPfOffQ + kPfNQ * kPfQTile;
-constexpr int kPfOffV = kPfOffK + kPfNSK * kPfKVTile;
-constexpr int kPfOffBar = kPfOffV + kPfNSV * kPfKVTile;
-// mbarriers: q, kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], vzero, drain, then
-// per Q tile: sfull (S ready), pready (P written), odone (the P V of the tile done)
-constexpr int kPfBarQ = 0, kPfBarKF = 1, kPfBarKE = kPfBarKF + kPfNSK, kPfBarVF = kPfBarKE + kPfNSK,
-              kPfBarVE = kPfBarVF + kPfNSV, kPfBarVZ = kPfBarVE + kPfNSV, kPfBarDrain = kPfBarVZ + 1,
-              kPfBarTile = kPfBarDrain + 1, kPfTileBars = 3, kPfBars = kPfBarTile + kPfTileBars * kPfNQ;
-constexpr int kPfOffSlot = kPfOffBar + kPfBars * 8;  // TMEM base address, abort flag
-constexpr int kPfOffML = kPfOffSlot + 16;            // (m, l) of slot 1 per row, for the split merge
-constexpr int kPfSmem = kPfOffML + 2 * kPfM * 4 + 1024;  // + room to align the base to 1024 B
+constexpr int kPfTileBars = 3;  // per Q tile: sfull (S ready), pready (P written), odone (its P V done)
+
+// Shared-memory layout. A bf16 pool streams V through three stages. An FP8
+// (E4M3) pool streams it through two, and the room of the third holds the
+// codes of one K tile and of one V tile as loaded, before the producer warps
+// widen them to f16 into the stages the MMA reads.
+template <bool FP8>
+struct PfLayout {
+    static constexpr int NSV = FP8 ? 2 : 3;  // V pipeline stages (a V tile is held longest)
+    static constexpr int OffV = kPfOffK + kPfNSK * kPfKVTile;
+    static constexpr int StgTile = kPfN * kPfD;  // E4M3 codes of one K or V tile: 16 KB
+    static constexpr int OffStg = OffV + NSV * kPfKVTile;
+    static constexpr int OffBar = OffStg + (FP8 ? 2 * StgTile : 0);
+    // mbarriers: q, kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], vzero, drain, the K and
+    // the V staging buffers (FP8: codes landed), q converted to f16 (FP8), then kPfTileBars
+    // per Q tile
+    static constexpr int BarQ = 0, BarKF = 1, BarKE = BarKF + kPfNSK, BarVF = BarKE + kPfNSK, BarVE = BarVF + NSV,
+                         BarVZ = BarVE + NSV, BarDrain = BarVZ + 1, BarStg = BarDrain + 1, BarQC = BarStg + 2,
+                         BarTile = BarQC + 1, Bars = BarTile + kPfTileBars * kPfNQ;
+    static constexpr int OffSlot = OffBar + Bars * 8;  // TMEM base address, abort flag
+    static constexpr int OffML = OffSlot + 16;         // (m, l) of slot 1 per row, for the split merge
+    static constexpr int Smem = OffML + 2 * kPfM * 4 + 1024;  // + room to align the base to 1024 B
+    static_assert(Smem <= 232448, "prefill shared memory over the 227 KB limit");
+    static_assert(OffStg % 1024 == 0 && StgTile % 1024 == 0, "staging and stages stay 1024-byte aligned");
+};
 // Tensor memory columns: S_A, S_B (128 fp32 each), then O_A, O_B (128 each). P of
 // a Q tile (128 bf16 = 64 columns) overwrites the first half of its own S.
 constexpr uint32_t kPfColP = 0;
@@ -256,7 +276,6 @@ constexpr uint32_t kPfColO = kPfNQ * kPfN;
 constexpr uint32_t kPfTmemCols = 512;
 constexpr int kPfBlocksPerTile = kPfN / kBlockSize;  // 8
 static_assert(kPfColO + kPfNQ * kPfD <= kPfTmemCols, "tensor memory over 512 columns");
-static_assert(kPfSmem <= 232448, "prefill shared memory over the 227 KB limit");
 static_assert(kPfBlocksPerTile <= 32, "one producer lane per block of a tile");
 
 struct PrefillParams {
@@ -270,7 +289,8 @@ struct PrefillParams {
     int num_kv_heads;
     int num_q_tokens;
     int num_seqs;
-    float scale_log2;
+    float scale_log2;  // softmax scale * log2(e) (times k_scale for an FP8 cache)
+    float v_scale;     // 1, or the FP8 value scale
 };
 
 // max(a, b, c) in one instruction (sm_100 has a three-input max)
@@ -280,9 +300,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// Two probabilities as the PV MMA's A operand: a bf16 pair, or an f16 pair
+// (F16), the first in the low half; and back.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_p(float p0, float p1) {
+    if constexpr (F16) {
+        const __half2 h = __floats2half2_rn(p0, p1);
+        return *reinterpret_cast<const uint32_t *>(&h);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+        return *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+template <bool F16>
+__device__ __forceinline__ void unpack_p(uint32_t u, float &p0, float &p1) {
+    if constexpr (F16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&u));
+        p0 = f.x;
+        p1 = f.y;
+    } else {
+        p0 = __uint_as_float(u << 16);
+        p1 = __uint_as_float(u & 0xffff0000u);
+    }
+}
+
 // p = 2^(x * sc + nm) for 64 scores of one row: the fp32 p are summed into acc
-// in packed pairs, and the bf16 pairs (keys 2w, 2w+1 in column w) are stored to
-// 32 TMEM columns at taddr.
+// in packed pairs, and the bf16 (F16: f16) pairs (keys 2w, 2w+1 in column w) are
+// stored to 32 TMEM columns at taddr.
+template <bool F16>
 __device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, float nm, f32x2 (&acc)[4],
                                             uint32_t taddr) {
     float pv[32];
@@ -295,13 +340,34 @@ __device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, floa
         const float p0 = ex2_approx(a0);
         const float p1 = ex2_approx(a1);
         add2(acc[w & 3], pack2(p0, p1));
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        pv[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
+        pv[w] = __uint_as_float(pack_p<F16>(p0, p1));
     }
     // finish the sums here: otherwise the compiler keeps the 64 p values alive
     // into the next half and runs out of registers
     asm volatile("" : "+l"(acc[0]), "+l"(acc[1]), "+l"(acc[2]), "+l"(acc[3]));
     tmem_st32(taddr, pv);
+}
+
+// Four E4M3 codes (low byte = element 0) to four f16 values, exactly (every
+// E4M3 value, subnormals included, is a normal f16 value or zero): two f16
+// pairs, element 0 in the low half of the first. One conversion per pair.
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t w) {
+    uint32_t lo, hi;
+    asm("{\n\t.reg .b16 c;\n\t"
+        "cvt.u16.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c;\n\t"
+        "cvt.u16.u32 c, %3;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w & 0xffffu), "r"(w >> 16));
+    return make_uint2(lo, hi);
+}
+
+// A bf16 pair to an f16 pair, rounded to nearest (exact for magnitudes in f16's
+// normal range and for zero).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // Work slots of a varlen launch: sequence b owns the slots starting at
@@ -347,10 +413,13 @@ __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, volatile 
     }
 }
 
-template <int G>
+// FP8: the caches hold E4M3 codes (values code * k_scale, code * v_scale);
+// q and out stay bf16.
+template <int G, bool FP8>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const PrefillParams prm, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    using L = PfLayout<FP8>;
     constexpr int TOK = kPfM / G;  // chunk tokens per Q tile
     constexpr int PER_CTA = kPfNQ * TOK;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -399,27 +468,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t raw_s = smem_addr(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
     unsigned char *base = smem_raw + (base_s - raw_s);
-    const uint32_t bars = base_s + kPfOffBar;
+    const uint32_t bars = base_s + L::OffBar;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * i; };
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kPfOffSlot);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + kPfOffSlot + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::OffSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L::OffSlot + 4);
 
     if (tid == 0) {
-        mbar_init(bar(kPfBarQ), 1);
+        mbar_init(bar(L::BarQ), 1);
         for (int i = 0; i < kPfNSK; ++i) {
-            mbar_init(bar(kPfBarKF + i), 1);
-            mbar_init(bar(kPfBarKE + i), 1);
+            mbar_init(bar(L::BarKF + i), 1);
+            mbar_init(bar(L::BarKE + i), 1);
         }
-        for (int i = 0; i < kPfNSV; ++i) {
-            mbar_init(bar(kPfBarVF + i), 1);
-            mbar_init(bar(kPfBarVE + i), 1);
+        for (int i = 0; i < L::NSV; ++i) {
+            mbar_init(bar(L::BarVF + i), 1);
+            mbar_init(bar(L::BarVE + i), 1);
         }
-        mbar_init(bar(kPfBarVZ), 1);
-        mbar_init(bar(kPfBarDrain), 1);
+        mbar_init(bar(L::BarVZ), 1);
+        mbar_init(bar(L::BarDrain), 1);
+        mbar_init(bar(L::BarStg), 1);      // FP8: K codes landed in the staging buffer
+        mbar_init(bar(L::BarStg + 1), 1);  // FP8: V codes landed
+        mbar_init(bar(L::BarQC), 2);  // FP8: both producer warps have converted their Q tile to f16
         for (int qi = 0; qi < kPfNQ; ++qi) {
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 0), 1);    // sfull: MMA commit
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 1), 128);  // pready: every softmax thread of the slot
-            mbar_init(bar(kPfBarTile + kPfTileBars * qi + 2), 1);    // odone: MMA commit
+            mbar_init(bar(L::BarTile + kPfTileBars * qi + 0), 1);    // sfull: MMA commit
+            mbar_init(bar(L::BarTile + kPfTileBars * qi + 1), 128);  // pready: every softmax thread of the slot
+            mbar_init(bar(L::BarTile + kPfTileBars * qi + 2), 1);    // odone: MMA commit
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -453,9 +525,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 return pb * kBlockSize;
             };
             const CUtensorMap *tm = is_v ? &tm_v : &tm_k;
-            const int ns = is_v ? kPfNSV : kPfNSK;
-            const uint32_t ring = base_s + (is_v ? kPfOffV : kPfOffK);
-            const int b_full = is_v ? kPfBarVF : kPfBarKF, b_empty = is_v ? kPfBarVE : kPfBarKE;
+            const int ns = is_v ? L::NSV : kPfNSK;
+            const uint32_t ring = base_s + (is_v ? L::OffV : kPfOffK);
+            const int b_full = is_v ? L::BarVF : L::BarKF, b_empty = is_v ? L::BarVE : L::BarKE;
             auto load_tile = [&](int s, int row) {
                 const uint32_t full = bar(b_full + s);
                 if (lane == 0) mbar_arrive_expect_tx(full, kPfKVTile);
@@ -467,53 +539,132 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
             };
             if (!is_v && lane == 0) {
-                mbar_arrive_expect_tx(bar(kPfBarQ), n_q * kPfQTile);
+                mbar_arrive_expect_tx(bar(L::BarQ), n_q * kPfQTile);
                 for (int qi = 0; qi < n_q; ++qi) {
                     const uint32_t dq = base_s + kPfOffQ + qi * kPfQTile;
                     const int qrow = q0 + t0 + qi * TOK;
-                    tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(kPfBarQ));
-                    tma_load_3d(dq + kPfQHalf, &tm_q, 64, hk * G, qrow, bar(kPfBarQ));
+                    tma_load_3d(dq, &tm_q, 0, hk * G, qrow, bar(L::BarQ));
+                    tma_load_3d(dq + kPfQHalf, &tm_q, 64, hk * G, qrow, bar(L::BarQ));
                 }
             }
-            int row = tile_row(0);
-            int issued = 0;
-            bool ok = true;
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                const int s = j % ns, u = j / ns;
-                const int row_next = tile_row(j + 1);  // fetched while this tile's loads go out
-                if (u >= 1) ok = pf_wait(bar(b_empty + s), (u - 1) & 1, abort_flag);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                load_tile(s, row);
-                issued = j + 1;
-                if (is_v && j == n_tiles - 1 && zero_tail) {
-                    // keys past the context: their V rows (tail slots) may hold anything, and
-                    // 0 * NaN would poison O, so zero them before the MMA reads the tile
-                    ok = __all_sync(0xffffffffu, pf_wait(bar(b_full + s), u & 1, abort_flag));
-                    if (ok) {
-                        const int first_bad = max(0, c - j * kPfN);
-                        unsigned char *vt = base + kPfOffV + s * kPfKVTile;
-                        for (int i = lane; i < (kPfN - first_bad) * 16; i += 32) {
-                            const int r = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
-                            *reinterpret_cast<uint4 *>(vt + half * kPfKVHalf + r * 128 + chunk * 16) =
-                                make_uint4(0, 0, 0, 0);
+            if constexpr (FP8) {
+                // The E4M3 codes of tile j land by TMA in this warp's staging buffer (16 rows
+                // x 128 B per block, row-major). The warp widens them to f16 into stage s, in
+                // the 128-byte-swizzled layout a TMA load of a 16-bit tile leaves (16-byte
+                // chunk k of row r at chunk k ^ (r % 8)), arrives on the stage's full barrier,
+                // and sends the next tile's codes, which load while the MMA works.
+                const uint32_t stg = base_s + L::OffStg + (is_v ? L::StgTile : 0);
+                const unsigned char *stg_p = base + L::OffStg + (is_v ? L::StgTile : 0);
+                const uint32_t b_stg = bar(L::BarStg + (is_v ? 1 : 0));
+                auto load_codes = [&](int rows) {  // this lane's block of the tile (lanes < 8)
+                    if (lane == 0) mbar_arrive_expect_tx(b_stg, L::StgTile);
+                    __syncwarp();
+                    if (lane < kPfBlocksPerTile) tma_load_3d(stg + lane * (kBlockSize * 128), tm, 0, hk, rows, b_stg);
+                };
+                int loaded = 1;  // code tiles sent to the staging buffer
+                load_codes(tile_row(0));
+                // while the first codes load: q to f16 in place (the MMAs take f16 operands
+                // here), Q tile 0 by the K producer, Q tile 1 (if any) by the V producer
+                const int qt = is_v ? 1 : 0;
+                if (qt < n_q) {
+                    const bool qok = __all_sync(0xffffffffu, pf_wait(bar(L::BarQ), 0, abort_flag));
+                    if (qok) {
+                        unsigned char *qp = base + kPfOffQ + qt * kPfQTile;
+#pragma unroll 4
+                        for (int i = lane; i < kPfQTile / 16; i += 32) {
+                            uint4 w = *reinterpret_cast<const uint4 *>(qp + i * 16);
+                            w = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z),
+                                           bf16x2_to_f16x2(w.w));
+                            *reinterpret_cast<uint4 *>(qp + i * 16) = w;
                         }
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bar(kPfBarVZ));
+                        fence_async_smem();  // the converted q to the MMA's proxy
                     }
                 }
-                row = row_next;
-            }
-            if (*abort_flag) {  // let loads nobody consumed land before the CTA exits
-                for (int i = 0; i < issued; ++i) mbar_wait(bar(b_full + i % ns), (i / ns) & 1);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::BarQC));
+                bool ok = true;
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    const int s = j % ns, u = j / ns;
+                    const int row_next = tile_row(j + 1);
+                    ok = pf_wait(b_stg, j & 1, abort_flag);
+                    if (ok && u >= 1) ok = pf_wait(bar(b_empty + s), (u - 1) & 1, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    // V rows past the context may hold any code (NaN included), and 0 * NaN
+                    // would poison O: they are written as zeros
+                    const int valid = is_v ? c - j * kPfN : kPfN;
+                    unsigned char *dst = base + (is_v ? L::OffV : kPfOffK) + s * kPfKVTile;
+#pragma unroll 4
+                    for (int it = 0; it < kPfN * 8 / 32; ++it) {
+                        const int i = it * 32 + lane, r = i / 8, c16 = i % 8;  // row r, codes 16 c16 .. + 15
+                        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+                        if (r < valid) {
+                            const uint4 w = *reinterpret_cast<const uint4 *>(stg_p + r * 128 + c16 * 16);
+                            const uint2 x0 = e4m3x4_to_f16x4(w.x), x1 = e4m3x4_to_f16x4(w.y);
+                            const uint2 x2 = e4m3x4_to_f16x4(w.z), x3 = e4m3x4_to_f16x4(w.w);
+                            lo = make_uint4(x0.x, x0.y, x1.x, x1.y);
+                            hi = make_uint4(x2.x, x2.y, x3.x, x3.y);
+                        }
+                        // dims 16 c16 .. + 15 are chunks 2 c16 % 8 and + 1 of half c16 / 4
+                        unsigned char *rp = dst + (c16 / 4) * kPfKVHalf + r * 128;
+                        const int k8 = (2 * c16) & 7;
+                        *reinterpret_cast<uint4 *>(rp + ((k8 ^ (r & 7)) * 16)) = lo;
+                        *reinterpret_cast<uint4 *>(rp + (((k8 + 1) ^ (r & 7)) * 16)) = hi;
+                    }
+                    // the widened tile to the MMA's (async) proxy, and the staging reads
+                    // ordered before the next TMA load overwrites the codes
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(b_full + s));
+                    if (j + 1 < n_tiles) {
+                        load_codes(row_next);
+                        loaded = j + 2;
+                    }
+                }
+                // a code load nobody widened lands before the CTA exits
+                if (*abort_flag) mbar_wait(b_stg, (loaded - 1) & 1);
+            } else {
+                int row = tile_row(0);
+                int issued = 0;
+                bool ok = true;
+                for (int j = 0; j < n_tiles && ok; ++j) {
+                    const int s = j % ns, u = j / ns;
+                    const int row_next = tile_row(j + 1);  // fetched while this tile's loads go out
+                    if (u >= 1) ok = pf_wait(bar(b_empty + s), (u - 1) & 1, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    load_tile(s, row);
+                    issued = j + 1;
+                    if (is_v && j == n_tiles - 1 && zero_tail) {
+                        // keys past the context: their V rows (tail slots) may hold anything, and
+                        // 0 * NaN would poison O, so zero them before the MMA reads the tile
+                        ok = __all_sync(0xffffffffu, pf_wait(bar(b_full + s), u & 1, abort_flag));
+                        if (ok) {
+                            const int first_bad = max(0, c - j * kPfN);
+                            unsigned char *vt = base + L::OffV + s * kPfKVTile;
+                            for (int i = lane; i < (kPfN - first_bad) * 16; i += 32) {
+                                const int r = first_bad + i / 16, half = (i / 8) & 1, chunk = i & 7;
+                                *reinterpret_cast<uint4 *>(vt + half * kPfKVHalf + r * 128 + chunk * 16) =
+                                    make_uint4(0, 0, 0, 0);
+                            }
+                            fence_async_smem();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(L::BarVZ));
+                        }
+                    }
+                    row = row_next;
+                }
+                if (*abort_flag) {  // let loads nobody consumed land before the CTA exits
+                    for (int i = 0; i < issued; ++i) mbar_wait(bar(b_full + i % ns), (i / ns) & 1);
+                }
             }
         } else if (warp == 1) {
             // ================= MMA issue (one thread) =================
             if (lane == 0) {
-                constexpr uint32_t kIdQK = idesc_bf16(kPfM, kPfN, 0);
-                constexpr uint32_t kIdPV = idesc_bf16(kPfM, kPfD, 1);
-                auto b_tile = [&](int qi, int k) -> uint32_t { return bar(kPfBarTile + kPfTileBars * qi + k); };
+                // an FP8 pool's tiles are widened to f16, so its MMAs take f16 operands
+                constexpr uint32_t kIdQK = idesc_f16kind(kPfM, kPfN, 0, FP8);
+                constexpr uint32_t kIdPV = idesc_f16kind(kPfM, kPfD, 1, FP8);
+                auto b_tile = [&](int qi, int k) -> uint32_t { return bar(L::BarTile + kPfTileBars * qi + k); };
                 // slot qi takes K/V tiles tile_of(qi, 0 .. n_of(qi) - 1); `last` marks the
                 // slot after whose MMA a K/V stage may be refilled
                 auto n_of = [&](int qi) -> int { return split ? (n_tiles - qi + 1) / 2 : n_tiles; };
@@ -526,29 +677,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     umma_qk_d128(tmem + qi * kPfN, smem_desc_sw128(qb, 16, 1024), smem_desc_sw128(kb, 16, 1024),
                                  kIdQK);
                     umma_commit(b_tile(qi, 0));
-                    if (last(qi)) umma_commit(bar(kPfBarKE + j % kPfNSK));
+                    if (last(qi)) umma_commit(bar(L::BarKE + j % kPfNSK));
                 };
                 auto issue_pv = [&](int qi, int j, bool acc) {  // O_qi (+)= P_qi V_j, P read from tensor memory
                     const uint32_t pt = tmem + qi * kPfN + kPfColP;
-                    const uint32_t vb = base_s + kPfOffV + (j % kPfNSV) * kPfKVTile;
+                    const uint32_t vb = base_s + L::OffV + (j % L::NSV) * kPfKVTile;
                     static_assert(kPfN == 128, "umma_pv_k128 covers 128 keys");
                     umma_pv_k128(tmem + kPfColO + qi * kPfD, pt, smem_desc_sw128(vb, kPfKVHalf, 1024), kIdPV,
                                  acc ? 1u : 0u);
                     umma_commit(b_tile(qi, 2));
-                    if (last(qi)) umma_commit(bar(kPfBarVE + j % kPfNSV));
+                    if (last(qi)) umma_commit(bar(L::BarVE + j % L::NSV));
                 };
                 // the first slot to read a K/V tile waits for it; in the unsplit order the
                 // second slot's MMA on the same tile comes after the first one's
                 auto wait_k = [&](int qi, int j) {
-                    return (qi > 0 && !split) || pf_wait(bar(kPfBarKF + j % kPfNSK), (j / kPfNSK) & 1, abort_flag);
+                    return (qi > 0 && !split) || pf_wait(bar(L::BarKF + j % kPfNSK), (j / kPfNSK) & 1, abort_flag);
                 };
                 auto wait_v = [&](int qi, int j) {
                     if (qi > 0 && !split) return true;
-                    return (j == n_tiles - 1 && zero_tail)
-                               ? pf_wait(bar(kPfBarVZ), 0, abort_flag)
-                               : pf_wait(bar(kPfBarVF + j % kPfNSV), (j / kPfNSV) & 1, abort_flag);
+                    // a bf16 pool's last tile is ready once its tail rows are zeroed; an FP8
+                    // pool's producer zeroes them while it widens the codes
+                    return (!FP8 && j == n_tiles - 1 && zero_tail)
+                               ? pf_wait(bar(L::BarVZ), 0, abort_flag)
+                               : pf_wait(bar(L::BarVF + j % L::NSV), (j / L::NSV) & 1, abort_flag);
                 };
-                bool ok = pf_wait(bar(kPfBarQ), 0, abort_flag);
+                bool ok = pf_wait(bar(FP8 ? L::BarQC : L::BarQ), 0, abort_flag);
                 for (int qi = 0; qi < n_slots && ok; ++qi) {
                     ok = wait_k(qi, tile_of(qi, 0));
                     if (!ok) break;
@@ -575,8 +728,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                 }
                 // every MMA issued so far completes before tensor memory can be freed
-                umma_commit(bar(kPfBarDrain));
-                mbar_wait(bar(kPfBarDrain), 0);
+                umma_commit(bar(L::BarDrain));
+                mbar_wait(bar(L::BarDrain), 0);
             }
             __syncwarp();
         } else {
@@ -586,9 +739,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int r = quad * 32 + lane;
             const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
             const uint32_t tS = tmem + qi * kPfN + lane_base, tO = tmem + kPfColO + qi * kPfD + lane_base;
-            const uint32_t b_sfull = bar(kPfBarTile + kPfTileBars * qi + 0);
-            const uint32_t b_pready = bar(kPfBarTile + kPfTileBars * qi + 1);
-            const uint32_t b_odone = bar(kPfBarTile + kPfTileBars * qi + 2);
+            const uint32_t b_sfull = bar(L::BarTile + kPfTileBars * qi + 0);
+            const uint32_t b_pready = bar(L::BarTile + kPfTileBars * qi + 1);
+            const uint32_t b_odone = bar(L::BarTile + kPfTileBars * qi + 2);
             const int tq = t0 + (split ? 0 : qi) * TOK;  // first chunk token of this slot's queries
             const int n_mine = split ? (n_tiles - qi + 1) / 2 : n_tiles;  // K/V tiles of this slot
             const int rows_valid = max(0, min(TOK, q_len - tq));
@@ -641,7 +794,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     };
                     auto exp_half = [&](f32x2 (&sum)[4], uint32_t col) {
                         // no unmasked key yet (m = -inf): every p is 0
-                        pf_exp_half(h, sl2, m_ref == -CUDART_INF_F ? -CUDART_INF_F : -m_ref, sum, tS + col);
+                        pf_exp_half<FP8>(h, sl2, m_ref == -CUDART_INF_F ? -CUDART_INF_F : -m_ref, sum, tS + col);
                     };
                     f32x2 acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc[4] = {0ull, 0ull, 0ull, 0ull};
                     load_half(0);
@@ -654,10 +807,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         tmem_ld32(tS, pa);
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
-                            const uint32_t u = __float_as_uint(pa[w]);
-                            const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(u << 16) * beta,
-                                                                            __uint_as_float(u & 0xffff0000u) * beta);
-                            pa[w] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pb));
+                            float p0, p1;
+                            unpack_p<FP8>(__float_as_uint(pa[w]), p0, p1);
+                            pa[w] = __uint_as_float(pack_p<FP8>(p0 * beta, p1 * beta));
                         }
                         tmem_st32(tS, pa);
                         const f32x2 b2 = pack2(beta, beta);
@@ -697,7 +849,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (split) {
                 // slot 1 hands (m, l) to slot 0 through shared memory; its O stays in TMEM,
                 // where slot 0's warps (same TMEM lanes) read it. All 8 softmax warps meet here.
-                float *ml = reinterpret_cast<float *>(base + kPfOffML);
+                float *ml = reinterpret_cast<float *>(base + L::OffML);
                 if (qi == 1) {
                     ml[r] = m_ref;
                     ml[kPfM + r] = l_sum;
@@ -716,7 +868,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (ok && active && (qi == 0 || !split)) {
                 tc_fence_after();
                 const bool row_ok = r / G < rows_valid;
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const float inv = l_sum > 0.f ? prm.v_scale / l_sum : 0.f;
                 const float ia = wa * inv, ib = wb * inv;
                 const uint32_t tOb = tmem + kPfColO + kPfD + lane_base;  // O of slot 1 (split only)
                 const int orow = row_ok ? q0 + tq + r / G : q0;
@@ -763,15 +915,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
 }
 
-template <int G>
+template <int G, bool FP8>
 int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cache, const void *v_cache,
                      int num_seqs, int max_q_len, int num_q_tokens, const pa_shape *s, cudaStream_t st) {
     constexpr int TOK = kPfM / G;
     CUtensorMap tm_q{}, tm_k{}, tm_v{};
     const uint64_t rows = static_cast<uint64_t>(s->num_blocks) * kBlockSize;
+    using L = PfLayout<FP8>;
+    // K/V boxes: a block's 16 rows of one KV head; bf16 as two 64-dim halves with the
+    // 128-byte swizzle the MMA reads, FP8 codes as whole 128-byte rows for the widening
+    const int ce = FP8 ? 1 : 2;
+    const uint32_t bx = FP8 ? kPfD : 64;
+    const CUtensorMapSwizzle sw = FP8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
     if (!encode_3d(&tm_q, q, kPfD, s->num_heads, num_q_tokens, 2, 64, G, TOK, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_3d(&tm_k, k_cache, kPfD, s->num_kv_heads, rows, 2, 64, 1, kBlockSize, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_3d(&tm_v, v_cache, kPfD, s->num_kv_heads, rows, 2, 64, 1, kBlockSize, CU_TENSOR_MAP_SWIZZLE_128B))
+        !encode_3d(&tm_k, k_cache, kPfD, s->num_kv_heads, rows, ce, bx, 1, kBlockSize, sw) ||
+        !encode_3d(&tm_v, v_cache, kPfD, s->num_kv_heads, rows, ce, bx, 1, kBlockSize, sw))
         return PA_ERR_UNSUPPORTED;
     // the shared-memory opt-in, once per device (bit per device; safe across host threads)
     static std::atomic<uint64_t> attr_done{0};
@@ -779,7 +937,7 @@ int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cach
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     const uint64_t bit = uint64_t{1} << (dev & 63);
     if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-        if (cudaFuncSetAttribute(prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem) !=
+        if (cudaFuncSetAttribute(prefill_kernel<G, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::Smem) !=
             cudaSuccess)
             return PA_ERR_CUDA;
         attr_done.fetch_or(bit, std::memory_order_acq_rel);
@@ -793,11 +951,11 @@ int launch_prefill_g(const PrefillParams &prm, const void *q, const void *k_cach
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(slots * s->num_kv_heads), 1, 1);
     cfg.blockDim = dim3(kPfThreads);
-    cfg.dynamicSmemBytes = kPfSmem;
+    cfg.dynamicSmemBytes = L::Smem;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<G>, prm, tm_q, tm_k, tm_v) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<G, FP8>, prm, tm_q, tm_k, tm_v) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 inline int launch_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -817,13 +975,24 @@ inline int launch_prefill(void *out, const void *q, const void *k_cache, const v
     prm.num_q_tokens = num_q_tokens;
     prm.num_seqs = num_seqs;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.v_scale = 1.f;
+    if (s->kv_fp8) {  // K = code * k_scale goes into the exponent's scale, V = code * v_scale into O's
+        prm.scale_log2 *= s->k_scale;
+        prm.v_scale = s->v_scale;
+    }
+#define PA_PREFILL_G(g)                                                                                           \
+    case g:                                                                                                       \
+        return s->kv_fp8                                                                                          \
+                   ? launch_prefill_g<g, true>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st) \
+                   : launch_prefill_g<g, false>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);
     switch (s->num_heads / s->num_kv_heads) {
-        case 1: return launch_prefill_g<1>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);
-        case 2: return launch_prefill_g<2>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);
-        case 4: return launch_prefill_g<4>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);
-        case 8: return launch_prefill_g<8>(prm, q, k_cache, v_cache, num_seqs, max_q_len, num_q_tokens, s, st);
+        PA_PREFILL_G(1)
+        PA_PREFILL_G(2)
+        PA_PREFILL_G(4)
+        PA_PREFILL_G(8)
         default: return PA_ERR_UNSUPPORTED;
     }
+#undef PA_PREFILL_G
 }
 
 }  // namespace pa

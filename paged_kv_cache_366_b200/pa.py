@@ -253,8 +253,9 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_
 
 
 def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_lens, max_q_len: int,
-                     scale: float, stream=None) -> None:
-    """Causal attention of query chunks at their context offsets (bf16, D=128)."""
+                     scale: float, stream=None, k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+    """Causal attention of query chunks at their context offsets (bf16 q/out, D=128; bf16 caches, or uint8
+    FP8 E4M3 caches with their k_scale / v_scale)."""
     _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(cu_q_lens, torch.int32, "cu_q_lens")
@@ -263,7 +264,7 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, cu_q_lens, context_
     B = context_lens.shape[0]
     if out.shape != q.shape or block_tables.shape[0] != B or cu_q_lens.shape[0] != B + 1:
         raise ValueError("q, out [T, H, D]; block_tables [B, MB]; cu_q_lens [B+1]; context_lens [B]")
-    shape = shape_of(k_cache, H)
+    shape = shape_of(k_cache, H, k_scale, v_scale)
     _check("pa_prefill_chunk",
            lib.pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                 block_tables.shape[1], _ptr(cu_q_lens), _ptr(context_lens), B, int(max_q_len), T,
