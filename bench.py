@@ -19,7 +19,8 @@ bandwidth, and against the nominal 8000 GB/s. `e2e` times the public
 DecodeStep API from pinned host buffers, with the copies inside.
 `cpu_baseline` is the fp64 oracle on the host cores. On the decode batch the
 line also carries, under `also`, the long-context decode, the prefill chunk,
-the FP8 pool, prefix sharing and a batch of verify chunks, each with its own
+decode and the chunk over an FP8 pool, prefix sharing, a batch of verify
+chunks, and the mixed step as two launches and as one, each with its own
 roofline and clocks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
@@ -359,9 +360,11 @@ def run_reference(args):
 ONE_LAUNCH = ("varlen_step", "spec_verify")
 NOMINAL_HBM_GBS = 8000.0  # the nominal HBM peak the targets are quoted against
 # Companions of the decode-batch line: the other target config (long context), the tensor-core
-# chunk, the FP8 pool, prefix sharing and a one-launch batch of verify chunks, each timed in the
-# same run with its own roofline and clocks.
-ALSO = ("long_context", "prefill_chunk", "decode_batch_fp8", "prefill_chunk_fp8", "prefix_sharing", "spec_verify")
+# chunk, the FP8 pool (decode and the chunk), prefix sharing, a one-launch batch of verify chunks,
+# and the mixed step as two launches and as one, each timed in the same run with its own roofline
+# and clocks.
+ALSO = ("long_context", "prefill_chunk", "decode_batch_fp8", "prefill_chunk_fp8", "prefix_sharing", "spec_verify",
+        "mixed_step", "varlen_step")
 
 
 def make_workload(name):
