@@ -20,8 +20,8 @@ DecodeStep API from pinned host buffers, with the copies inside.
 `cpu_baseline` is the fp64 oracle on the host cores. On the decode batch the
 line also carries, under `also`, the long-context decode, the prefill chunk,
 decode and the chunk over an FP8 pool, prefix sharing, a batch of verify
-chunks, and the mixed step as two launches and as one, each with its own
-roofline and clocks.
+chunks, the mixed step as two launches and as one, and the block copy and
+swap, each with its own roofline and clocks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
@@ -726,6 +726,10 @@ def run_ours(args):
                 ent["unique_bytes"] = unique_bytes_entry(mx, peak)
             also[extra] = ent
             del mx
+        for extra in BLOCK_WORKLOADS:
+            torch.cuda.empty_cache()
+            bl = measure_blocks(extra, max(5, min(args.steps, 50)), args.warmup, sampler)
+            also[extra] = {k: bl[k] for k in ("steps", "ms_per_step", "value", "unit", "clocks", "config", "roofline")}
 
     if world > 1:
         dist.destroy_process_group()
@@ -786,7 +790,15 @@ def run_ours(args):
 
 
 def run_blocks(args):
-    """Whole-block copies on the decode-batch pool.
+    """Whole-block copies on the decode-batch pool (see measure_blocks): one JSON line."""
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
+        return 0  # replicas of a copy measure nothing the single run does not
+    print(json.dumps(measure_blocks(args.workload, args.steps, args.warmup)), flush=True)
+    return 0
+
+
+def measure_blocks(workload, steps, warmup, sampler=None):
+    """Whole-block copies on the decode-batch pool; returns the bench line.
 
     copy_blocks: copy-on-write of 2048 (used -> free) blocks, K and V, inside HBM.
     swap_blocks: 2048 blocks of K and V out to pinned host memory and back in,
@@ -795,8 +807,6 @@ def run_blocks(args):
     import torch
     from paged_kv_cache_366_b200 import pa
 
-    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
-        return 0  # replicas of a copy measure nothing the single run does not
     case = W.decode_batch()
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
     k_cache, v_cache = dev(case.k_cache), dev(case.v_cache)
@@ -808,7 +818,7 @@ def run_blocks(args):
     stream = torch.cuda.Stream()
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    if args.workload == "copy_blocks":
+    if workload == "copy_blocks":
         pairs = torch.from_numpy(np.stack([rng.choice(used, n), rng.choice(free, n, replace=False)], 1)
                                  .astype(np.int64)).cuda()
         fns = [lambda: pa.pa_copy_blocks(k_cache, v_cache, pairs)]
@@ -852,16 +862,18 @@ def run_blocks(args):
         with torch.cuda.graph(g, stream=stream):
             for f in fns:
                 f()
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             flush_w.zero_()
             torch.sum(flush_r)
             g.replay()
     torch.cuda.synchronize()
     if pa.pa_get_status(stream):
         raise SystemExit("device status set by the block copies")
-    sampler = ClockSampler(gpu_id_for(int(os.environ.get("LOCAL_RANK", "0"))))
-    sampler.wait_ready()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    own_sampler = sampler is None
+    if own_sampler:
+        sampler = ClockSampler(gpu_id_for(int(os.environ.get("LOCAL_RANK", "0"))))
+        sampler.wait_ready()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     wall0 = time.time()
     with torch.cuda.stream(stream):
         for a, b in ev:
@@ -872,21 +884,21 @@ def run_blocks(args):
             b.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
-    sampler.stop()
-    t = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / args.steps
+    clocks = sampler.window(wall0, wall1)
+    if own_sampler:
+        sampler.stop()
+    del g
+    t = sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / steps
     value = nbytes / t / 1e9
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; see paged_kv_cache_366_b200/workloads.py)",
-            "config": {"workload": args.workload, "pool": "decode_batch (seed 1)", "block_pairs": n,
+            "config": {"workload": workload, "pool": "decode_batch (seed 1)", "block_pairs": n,
                        "block_bytes_per_pool": block_bytes,
                        "l2": "flushed before every step, outside the events (memset then read)"},
             "roofline": {"bound": bound, "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
                          "traffic": None, "kernel": "copy_blocks_kernel", "peak_kind": peak_note},
-            "cpu_baseline": None, "e2e": None, "clocks": sampler.window(wall0, wall1),
-            "gpu_launches": launches * args.steps}
-    print(json.dumps(line), flush=True)
-    return 0
+            "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": launches * steps}
 
 
 def main(argv=None):
