@@ -14,7 +14,8 @@
 //    K/V tile loaded serves all G heads of both Q tiles. A chunk too short to
 //    reach the second tile (a decode token, a short verify chunk) runs one.
 //  * Warp 0 streams Q and then 128-key K tiles by TMA with 128-byte swizzle
-//    into a 2-stage ring, and warp 10 the V tiles into a 3-stage ring, so
+//    into a 2-stage ring, and warp 10 the V tiles into a 3-stage ring (2 over
+//    an FP8 pool), so
 //    neither load waits behind the other's free stage. A tile is eight 16-token
 //    blocks, and each block of each 64-column half is one TMA box addressed
 //    through the block table. Blocks past the context (and bad table entries) load from an
