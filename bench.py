@@ -377,18 +377,6 @@ def make_workload(name):
     return W.CONFIGS[name]()
 
 
-def blocks_unshared(case, seqs):
-    """True when no physical block holds context of two of `seqs` (the kv_unshared hint's condition)."""
-    seen = set()
-    for b in seqs:
-        nblk = (int(case.context_lens[b]) + case.block_size - 1) // case.block_size
-        for pb in case.block_tables[b, :nblk]:
-            if int(pb) in seen:
-                return False
-            seen.add(int(pb))
-    return True
-
-
 def unique_kv_bytes(case, dec):
     """K/V bytes of the distinct physical rows the decode sequences read (shared blocks counted once)."""
     Hk, D, E = case.num_kv_heads, case.head_dim, case.elem_bytes
@@ -459,7 +447,6 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
     max_ctx = int(case.context_lens[dec].max()) if len(dec) else 0
     ws_n = pa.pa_decode_workspace_bytes(len(dec), max_ctx, 0, shape) if len(dec) else 0
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda") if ws_n else None
-    unshared = bool(len(dec)) and blocks_unshared(case, dec)  # decided from the tables, as an engine would
 
     if len(pre):
         p0, p1 = int(pre[0]), int(pre[-1]) + 1
@@ -476,15 +463,15 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
 
     def do_decode():  # the partition pass, then the merge of cut units (a programmatic dependent)
         pa.pa_decode(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0, ws,
-                     k_scale=ks, v_scale=vs, kv_unshared=unshared)
+                     k_scale=ks, v_scale=vs)
 
     def do_partials():  # the partition pass alone: decode_kernel, the dominant kernel
         pa.pa_decode_partials(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0,
-                              ws, k_scale=ks, v_scale=vs, kv_unshared=unshared)
+                              ws, k_scale=ks, v_scale=vs)
 
     def do_merge():  # the merge alone, on the partials the pass before it left in the workspace
         pa.pa_decode_merge(out_dec, q_dec, k_cache, v_cache, tables[d0:d1], lens[d0:d1], max_ctx, case.scale, 0,
-                           ws, k_scale=ks, v_scale=vs, kv_unshared=unshared)
+                           ws, k_scale=ks, v_scale=vs)
 
 
     def do_prefill():
@@ -579,7 +566,7 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
     e2e = None
     if want_e2e and len(dec) and not len(pre):
         step = DecodeStep(k_cache, v_cache, case.num_heads, len(dec), case.max_blocks_per_seq, max_ctx,
-                          case.scale, k_scale=ks, v_scale=vs, kv_unshared=unshared)
+                          case.scale, k_scale=ks, v_scale=vs)
         rows = np.asarray([int(case.cu_q_lens[b + 1]) - 1 for b in dec], np.int64)
         views = step.inputs()  # staged inputs: the step's six inputs in one pinned buffer
 
@@ -614,7 +601,7 @@ def measure_gpu(name, steps, warmup, flush, sampler, want_e2e):
                "api": "paged_kv_cache_366_b200.step.DecodeStep, staged inputs (one copy in, one out; CUDA graph)"}
     del graphs, g_step
     return {"case": case, "dec": dec, "pre": pre, "nbytes": nbytes, "total": total, "per_part": per_part,
-            "clocks": clocks, "e2e": e2e, "one": one, "fp8": fp8, "ks": ks, "vs": vs, "unshared": unshared,
+            "clocks": clocks, "e2e": e2e, "one": one, "fp8": fp8, "ks": ks, "vs": vs,
             "launches_per_step": launches_per_step, "wall": (wall0, wall1)}
 
 
@@ -767,8 +754,6 @@ def run_ours(args):
         cpu.pop("n_seqs", None)
     parts_ms = {k: v * 1e3 for k, v in per_part.items()}
     config = describe(case, dec, pre)
-    if len(dec):
-        config["kv_unshared"] = m["unshared"]  # the decode hint, decided from the tables
     if m["fp8"]:
         config.update({"workload": args.workload, "kv_dtype": "fp8_e4m3", "k_scale": m["ks"],
                        "v_scale": m["vs"]})

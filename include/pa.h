@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 6
+#define PA_ABI_VERSION 7
 #define PA_BLOCK_SIZE 16
 
 typedef enum {
@@ -100,15 +100,6 @@ typedef struct {
     int32_t kv_fp8;
     float k_scale; /* > 0 when kv_fp8; ignored otherwise */
     float v_scale; /* > 0 when kv_fp8; ignored otherwise */
-    /*
-     * Decode only, a hint (0 or 1): 1 says that no cache block appears in the
-     * tables of two sequences of this call (no shared prefix), so each K/V
-     * block is read once. Decode then marks K/V lines first to evict in L2
-     * when the longest context is at most 4096 tokens, keeping its partials,
-     * queries and tables there. Results are the same either way; a wrong 1
-     * only costs re-reads of shared blocks.
-     */
-    int32_t kv_unshared;
 } pa_shape;
 
 /*

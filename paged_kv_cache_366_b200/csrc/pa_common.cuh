@@ -105,6 +105,13 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
+// The normal L2 eviction priority as an explicit policy (createpolicy result).
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 // ---- arithmetic ---------------------------------------------------------------
 
 // Packed pairs of fp32 in one 64-bit register, for the two-wide fp32 ops

@@ -25,7 +25,7 @@ PA_STATUS_BAD_SLOT = 0x2
 PA_STATUS_BAD_CONTEXT = 0x4
 PA_STATUS_WAIT_TIMEOUT = 0x8
 PA_STATUS_BAD_QUERY = 0x10
-PA_ABI_VERSION = 6
+PA_ABI_VERSION = 7
 
 
 class PaShape(ctypes.Structure):
@@ -39,7 +39,6 @@ class PaShape(ctypes.Structure):
         ("kv_fp8", ctypes.c_int32),
         ("k_scale", ctypes.c_float),
         ("v_scale", ctypes.c_float),
-        ("kv_unshared", ctypes.c_int32),
     ]
 
 
@@ -130,13 +129,11 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError("dtype must be bfloat16 or float32, got %s" % dt)
 
 
-def shape_of(k_cache: torch.Tensor, num_heads: int, k_scale: float = 0.0, v_scale: float = 0.0,
-             kv_unshared: bool = False) -> PaShape:
+def shape_of(k_cache: torch.Tensor, num_heads: int, k_scale: float = 0.0, v_scale: float = 0.0) -> PaShape:
     """pa_shape of a pool [NB, 16, Hk, D] read by `num_heads` query heads.
 
     A uint8 pool holds FP8 E4M3 codes (values code * k_scale / code * v_scale)
-    next to bf16 q/out and new tokens. kv_unshared: the caller's word that no
-    block appears in two sequences' tables of the call (a decode hint).
+    next to bf16 q/out and new tokens.
     """
     if k_cache.dim() != 4:
         raise ValueError("k_cache must be [num_blocks, block_size, num_kv_heads, head_dim]")
@@ -144,8 +141,7 @@ def shape_of(k_cache: torch.Tensor, num_heads: int, k_scale: float = 0.0, v_scal
     fp8 = k_cache.dtype == torch.uint8
     return PaShape(num_heads=int(num_heads), num_kv_heads=int(hk), head_dim=int(d), block_size=int(bs),
                    num_blocks=int(nb), dtype=PA_DTYPE_BF16 if fp8 else _dtype_code(k_cache.dtype),
-                   kv_fp8=1 if fp8 else 0, k_scale=float(k_scale), v_scale=float(v_scale),
-                   kv_unshared=1 if kv_unshared else 0)
+                   kv_fp8=1 if fp8 else 0, k_scale=float(k_scale), v_scale=float(v_scale))
 
 
 def _same_dtype_kv(q_like, caches):
@@ -192,14 +188,14 @@ def pa_decode_workspace_bytes(num_seqs: int, max_context_len: int, partition_tok
 
 
 def _decode(fn: str, out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale, kv_unshared) -> None:
+            partition_tokens, workspace, stream, k_scale, v_scale) -> None:
     _same_dtype_kv((out, q), (k_cache, v_cache))
     _int(block_tables, torch.int32, "block_tables")
     _int(context_lens, torch.int32, "context_lens")
     B, H, D = q.shape
     if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
-    shape = shape_of(k_cache, H, k_scale, v_scale, kv_unshared)
+    shape = shape_of(k_cache, H, k_scale, v_scale)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(fn,
            getattr(lib, fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
@@ -210,33 +206,30 @@ def _decode(fn: str, out, q, k_cache, v_cache, block_tables, context_lens, max_c
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
               partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-              k_scale: float = 0.0, v_scale: float = 0.0, kv_unshared: bool = False) -> None:
-    """Decode attention of one query token per sequence over its paged context.
-
-    kv_unshared=True: no block appears in two sequences' tables (see pa_shape.kv_unshared)."""
+              k_scale: float = 0.0, v_scale: float = 0.0) -> None:
+    """Decode attention of one query token per sequence over its paged context."""
     _decode("pa_decode", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale, kv_unshared)
+            partition_tokens, workspace, stream, k_scale, v_scale)
 
 
 def pa_decode_partials(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
                        partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-                       k_scale: float = 0.0, v_scale: float = 0.0, kv_unshared: bool = False) -> None:
+                       k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """The first of pa_decode's two launches: the partition pass (arguments as pa_decode)."""
     _decode("pa_decode_partials", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale, kv_unshared)
+            partition_tokens, workspace, stream, k_scale, v_scale)
 
 
 def pa_decode_merge(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
                     partition_tokens: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
-                    k_scale: float = 0.0, v_scale: float = 0.0, kv_unshared: bool = False) -> None:
+                    k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """The second of pa_decode's two launches: the merge of cut units (arguments as pa_decode)."""
     _decode("pa_decode_merge", out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
-            partition_tokens, workspace, stream, k_scale, v_scale, kv_unshared)
+            partition_tokens, workspace, stream, k_scale, v_scale)
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float,
-                      partition_tokens: int = 0, stream=None, k_scale: float = 0.0, v_scale: float = 0.0,
-                      kv_unshared: bool = False) -> None:
+                      partition_tokens: int = 0, stream=None, k_scale: float = 0.0, v_scale: float = 0.0) -> None:
     """pa_decode without a workspace argument, for callers that cannot allocate device memory.
 
     The split-context partials go to a PA_NOALLOC_SCRATCH_BYTES array built
@@ -252,7 +245,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, max_
     B, H, D = q.shape
     if out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise ValueError("q, out [B, H, D]; block_tables [B, MB]; context_lens [B]")
-    shape = shape_of(k_cache, H, k_scale, v_scale, kv_unshared)
+    shape = shape_of(k_cache, H, k_scale, v_scale)
     _check("pa_decode_noalloc",
            lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(context_lens), B, int(max_context_len), float(scale),

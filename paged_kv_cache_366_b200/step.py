@@ -31,12 +31,11 @@ _ALIGN = 256  # byte alignment of each input inside the staging buffers
 class DecodeStep:
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_heads: int, num_seqs: int,
                  max_blocks_per_seq: int, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 use_graph: bool = True, k_scale: float = 0.0, v_scale: float = 0.0, kv_unshared: bool = False):
+                 use_graph: bool = True, k_scale: float = 0.0, v_scale: float = 0.0):
         if not (k_cache.is_cuda and v_cache.is_cuda):
             raise ValueError("the KV pool lives on the device")
         self.k_cache, self.v_cache = k_cache, v_cache
         self.k_scale, self.v_scale = k_scale, v_scale  # for a uint8 (FP8 E4M3) pool
-        self.kv_unshared = kv_unshared  # no block in two sequences' tables (pa_shape.kv_unshared)
         dev = k_cache.device
         dt = torch.bfloat16 if k_cache.dtype == torch.uint8 else k_cache.dtype
         _, _, hk, d = k_cache.shape
@@ -114,7 +113,7 @@ class DecodeStep:
                                 k_scale=self.k_scale, v_scale=self.v_scale)
         pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                      self.max_context_len, self.scale, self.partition_tokens, self.workspace,
-                     k_scale=self.k_scale, v_scale=self.v_scale, kv_unshared=self.kv_unshared)
+                     k_scale=self.k_scale, v_scale=self.v_scale)
         self._result().copy_(self.out, non_blocking=True)
 
     def _result(self) -> torch.Tensor:

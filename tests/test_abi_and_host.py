@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_messages():
     from paged_kv_cache_366_b200 import pa
-    assert pa.pa_abi_version() == 6
+    assert pa.pa_abi_version() == 7
     assert pa.pa_strerror(0) == "ok"
     assert "workspace" in pa.pa_strerror(-4)
     assert pa.pa_strerror(-99) == "unknown error"
@@ -97,7 +97,7 @@ def test_shape_validation(kw, code):
 @pytest.mark.parametrize("kw,code", [
     (dict(kv_fp8=1, k_scale=0.1, v_scale=0.1), 0), (dict(kv_fp8=1, k_scale=0.0, v_scale=0.1), -1),
     (dict(kv_fp8=1, k_scale=0.1, v_scale=float("inf")), -1), (dict(kv_fp8=1, dtype=0, k_scale=1.0, v_scale=1.0), -2),
-    (dict(kv_fp8=2), -1), (dict(kv_unshared=1), 0), (dict(kv_unshared=2), -1),
+    (dict(kv_fp8=2), -1),
 ])
 def test_fp8_cache_shape_validation(kw, code):
     from paged_kv_cache_366_b200 import pa

@@ -23,7 +23,7 @@ def pa():
     return _pa
 
 
-def run_step(pa, case, seqs=None, partition_tokens=0, dev=None, kv_unshared=False):
+def run_step(pa, case, seqs=None, partition_tokens=0, dev=None):
     """Write this step's tokens, then decode `seqs` (default: all). Returns (out, k_cache, v_cache, status)."""
     d = dev or DevCase(case)
     pa.pa_reshape_and_cache(d.k_new, d.v_new, d.k_cache, d.v_cache, d.slot_mapping)
@@ -39,8 +39,7 @@ def run_step(pa, case, seqs=None, partition_tokens=0, dev=None, kv_unshared=Fals
     shape = pa.shape_of(d.k_cache, case.num_heads)
     nbytes = pa.pa_decode_workspace_bytes(len(seqs), max_ctx, partition_tokens, shape)
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda") if nbytes else None
-    pa.pa_decode(out, q, d.k_cache, d.v_cache, bt, cl, max_ctx, case.scale, partition_tokens, ws,
-                 kv_unshared=kv_unshared)
+    pa.pa_decode(out, q, d.k_cache, d.v_cache, bt, cl, max_ctx, case.scale, partition_tokens, ws)
     status = pa.pa_get_status()
     return out, d.k_cache, d.v_cache, status
 
@@ -204,17 +203,6 @@ def test_decode_is_deterministic(pa):
     a, *_ = run_step(pa, case)
     b, *_ = run_step(pa, case)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
-
-
-def test_unshared_hint_changes_nothing_but_the_cache_policy(pa):
-    # the decode batch (no shared block, contexts up to 2048: the hint takes effect) and a long
-    # ragged list past the hint's context limit: bit-identical outputs with and without it
-    for case in (W.decode_batch(), W.make_case("hint", 6, context_lens=[5000, 700, 33], q_lens=[1, 1, 1],
-                                               num_heads=32, num_kv_heads=8, head_dim=128, dtype="bf16")):
-        a, *_ , sa = run_step(pa, case)
-        b, *_ , sb = run_step(pa, case, kv_unshared=True)
-        assert sa == 0 and sb == 0
-        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 def test_negative_slot_is_skipped(pa):
