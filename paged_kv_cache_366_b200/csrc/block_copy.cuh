@@ -31,7 +31,20 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ ds
         }
         const uint4 *sp = src + s * block_vecs;
         uint4 *dp = dst + d * block_vecs;
-        for (int v = threadIdx.x; v < block_vecs; v += blockDim.x) dp[v] = __ldcs(sp + v);
+        // eight loads of each thread in flight before its stores (a 32 KB block is 8 per thread)
+        for (int v0 = threadIdx.x; v0 < block_vecs; v0 += 8 * blockDim.x) {
+            uint4 r[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int v = v0 + u * blockDim.x;
+                if (v < block_vecs) r[u] = __ldcs(sp + v);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int v = v0 + u * blockDim.x;
+                if (v < block_vecs) __stcs(dp + v, r[u]);
+            }
+        }
     }
 }
 
